@@ -1,0 +1,42 @@
+// kernels.h -- internal launchers of libmsa (host side).  Not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "msa_common.cuh"
+
+namespace msa {
+
+// SIMT kernels (kernels_simt.cu)
+cudaError_t launch_decode_index(const Shape &sh, const void *q_idx, const void *k_idx,
+                                int32_t *ids, float *block_scores, int num_sms, cudaStream_t st);
+size_t decode_attn_smem_bytes(const Shape &sh);
+cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, const void *v,
+                               const int32_t *ids, float *part_o, float *part_lse, int S,
+                               int *status, cudaStream_t st);
+cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
+                           const float *part_lse, const int32_t *ids, float *out, float *lse,
+                           int S, cudaStream_t st);
+cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts,
+                          int *pair_totals, int32_t *row_ptr, int32_t *entries, int *item_ptr,
+                          AttnItem *items, int *counters, int rows_per_item, int n_chunks,
+                          int *status, cudaStream_t st);
+
+// tcgen05 kernels (kernels_tc.cu)
+size_t selftest_smem_bytes(int N, int Kd);
+cudaError_t launch_selftest_umma(const CUtensorMap &tm_a, const CUtensorMap &tm_b, float *C,
+                                 int N, int Kd, int b_mn_major, int *status, cudaStream_t st);
+size_t prefill_index_smem_bytes(int d_idx);
+cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                 int32_t *ids, int *status, int num_sms, cudaStream_t st);
+size_t prefill_attn_smem_bytes(const Shape &sh);
+cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                                const void *q, const int32_t *row_ptr, const int32_t *entries,
+                                const AttnItem *items, int *counters, void *part_o,
+                                float *part_lse, int *status, int num_sms, cudaStream_t st);
+
+}  // namespace msa

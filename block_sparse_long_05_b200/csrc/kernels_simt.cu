@@ -1,0 +1,653 @@
+// kernels_simt.cu -- the HBM-bound and integer kernels of the MSA hot path:
+//   * decode index scan + top-K select  (index branch, one query per sequence)
+//   * split-K decode attention           (sparse branch, one query per sequence)
+//   * log-sum-exp combine of partials    (prefill and decode)
+//   * selection inversion (CSR of hit queries per KV block)
+//
+// Method: "MiniMax M3模型算力成本大幅降低原因深度解析" (index branch: single-head
+// index key, block max-pool, top-K; sparse branch: GQA over the kept blocks)
+// and "MiniMax M3 深度实战", sections 2.2 (KV outer gather Q: per-block hit
+// lists), 2.3 (softmax(QK^T/sqrt(d))V over gathered keys) and 3.3 (decode).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cstdint>
+
+#include "kernels.h"
+#include "msa_common.cuh"
+
+namespace msa {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// Total order on (score desc, block asc) packed into 64 bits: larger key
+// ranks first.  Scores are finite.
+__device__ __forceinline__ uint64_t rank_key(float s, int j) {
+    uint32_t u = __float_as_uint(s);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(0x7FFFFFFF - j);
+}
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+    uint32_t lo = static_cast<uint32_t>(v), hi = static_cast<uint32_t>(v >> 32);
+    lo = __shfl_xor_sync(0xFFFFFFFFu, lo, m);
+    hi = __shfl_xor_sync(0xFFFFFFFFu, hi, m);
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// ------------------------------------------------------------------------
+// Decode index scan: block_scores[b][j] = max_{i in block j} q_idx[b].k_idx[b][i]
+// for j < own = (T-1)/block.  One warp per (b, j); 16-byte streaming loads,
+// D_IDX/8 lanes per key row.  fp32 accumulation (exact for integer keys).
+// ------------------------------------------------------------------------
+template <int D_IDX>
+__global__ void __launch_bounds__(256) decode_index_scan_kernel(
+    const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16 *__restrict__ k_idx,
+    float *__restrict__ block_scores, int Bt, int T, int block, int own, int N) {
+    constexpr int LPR = D_IDX / 8;  // lanes per key row
+    constexpr int RPL = 32 / LPR;   // key rows per warp load
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / LPR;
+    const int part = lane % LPR;
+    const long long warps_total = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+    const long long work = static_cast<long long>(Bt) * own;
+    int cur_b = -1;
+    float qv[8];
+    for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+         w < work; w += warps_total) {
+        const int b = static_cast<int>(w / own);
+        const int j = static_cast<int>(w % own);
+        if (b != cur_b) {
+            const uint4 qu =
+                *reinterpret_cast<const uint4 *>(q_idx + static_cast<long long>(b) * D_IDX + part * 8);
+            bf16x8_to_f32(qu, qv);
+            cur_b = b;
+        }
+        const uint4 *base = reinterpret_cast<const uint4 *>(
+            k_idx + (static_cast<long long>(b) * T + static_cast<long long>(j) * block) * D_IDX);
+        float best = -FLT_MAX;
+        const int iters = block / RPL;
+#pragma unroll 8
+        for (int it = 0; it < iters; ++it) {
+            const int r = sub + RPL * it;
+            const uint4 ku = __ldcs(base + r * LPR + part);
+            float kf[8];
+            bf16x8_to_f32(ku, kf);
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s = fmaf(qv[e], kf[e], s);
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+            best = fmaxf(best, s);
+        }
+#pragma unroll
+        for (int o = LPR; o < 32; o <<= 1) best = fmaxf(best, __shfl_xor_sync(0xFFFFFFFFu, best, o));
+        if (lane == 0) block_scores[static_cast<long long>(b) * N + j] = best;
+    }
+}
+
+// ------------------------------------------------------------------------
+// Decode select: one warp per sequence.  Each lane keeps a sorted top list of
+// its strided candidates, then min(K, own+1)-1 rounds of warp arg-max over
+// the lanes' heads pick the winners; own is added and ids written ascending.
+// ------------------------------------------------------------------------
+template <int CAP>
+__global__ void __launch_bounds__(32) decode_select_kernel(const float *__restrict__ block_scores,
+                                                           int32_t *__restrict__ ids, int N,
+                                                           int own, int K) {
+    const int b = blockIdx.x;
+    const int lane = threadIdx.x;
+    uint64_t top[CAP];
+#pragma unroll
+    for (int p = 0; p < CAP; ++p) top[p] = 0;  // 0 ranks below every real key
+    for (int j = lane; j < own; j += 32) {
+        uint64_t key = rank_key(block_scores[static_cast<long long>(b) * N + j], j);
+        if (key > top[CAP - 1]) {
+            bool ins = false;
+#pragma unroll
+            for (int p = 0; p < CAP; ++p) {
+                const bool take = ins || key > top[p];
+                if (take) {
+                    const uint64_t t = top[p];
+                    top[p] = key;
+                    key = t;
+                    ins = true;
+                }
+            }
+        }
+    }
+    const int m = min(K, own + 1) - 1;
+    __shared__ int sel[kMaxK];
+    for (int p = 0; p < m; ++p) {
+        uint64_t best = top[0];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint64_t other = shfl_xor_u64(best, o);
+            best = other > best ? other : best;
+        }
+        if (top[0] == best && best != 0) {  // keys are unique: exactly one lane pops
+#pragma unroll
+            for (int q = 0; q < CAP - 1; ++q) top[q] = top[q + 1];
+            top[CAP - 1] = 0;
+        }
+        if (lane == 0) sel[p] = 0x7FFFFFFF - static_cast<int>(static_cast<uint32_t>(best));
+    }
+    __syncwarp();
+    if (lane == 0) {
+        sel[m] = own;
+        const int n = m + 1;
+        for (int a = 1; a < n; ++a) {  // insertion sort, ascending
+            const int x = sel[a];
+            int c = a - 1;
+            while (c >= 0 && sel[c] > x) {
+                sel[c + 1] = sel[c];
+                --c;
+            }
+            sel[c + 1] = x;
+        }
+        for (int s = 0; s < K; ++s) ids[static_cast<long long>(b) * K + s] = s < n ? sel[s] : -1;
+    }
+}
+
+// ------------------------------------------------------------------------
+// Split-K decode attention.  One CTA per (b, kv head, slot, split of
+// kDecodeKeys keys).  K/V rows staged in shared memory by 16-byte cp.async
+// (coalesced 2*d-byte rows), G query heads share them; fp32 softmax in the
+// log2 domain.  Writes a normalised fp32 partial and its natural-log lse
+// (-inf when the split has no key).
+// ------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) decode_attn_kernel(
+    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+    const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ ids,
+    float *__restrict__ part_o, float *__restrict__ part_lse, int T, int Hq, int Hkv, int block,
+    int K, int S, int N, float scale_log2, int *__restrict__ status) {
+    constexpr int KS = kDecodeKeys;
+    constexpr int KSTR = D + 8;  // padded K row (bf16) to spread banks
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int G = Hq / Hkv;
+    float *qs = reinterpret_cast<float *>(smem_raw);                       // [G][D]
+    float *ps = qs + G * D;                                                 // [G][KS]
+    float *ms = ps + G * KS;                                                // [G]
+    float *ls = ms + G;                                                     // [G]
+    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(
+        (reinterpret_cast<uintptr_t>(ls + G) + 15) & ~static_cast<uintptr_t>(15));  // [KS][KSTR]
+    __nv_bfloat16 *Vs = Ks + KS * KSTR;                                     // [KS][D]
+
+    const int tid = threadIdx.x;
+    int idx = blockIdx.x;
+    const int p = idx % S;
+    idx /= S;
+    const int s = idx % K;
+    idx /= K;
+    const int hk = idx % Hkv;
+    const int b = idx / Hkv;
+    const long long prow = (static_cast<long long>(b) * K + s) * S + p;  // partial row
+    const int t = T - 1;
+    const int j = ids[static_cast<long long>(b) * K + s];
+    int nk = 0;
+    long long k0 = 0;
+    if (j >= N || j < -1) {
+        if (tid == 0) atomicOr(status, kDevBadIds);
+    } else if (j >= 0) {
+        k0 = static_cast<long long>(j) * block + static_cast<long long>(p) * KS;
+        long long k1 = k0 + KS;
+        const long long blk_end = static_cast<long long>(j + 1) * block;
+        if (k1 > blk_end) k1 = blk_end;
+        if (k1 > T) k1 = T;
+        if (k1 > t + 1) k1 = t + 1;
+        nk = k1 > k0 ? static_cast<int>(k1 - k0) : 0;
+    }
+    if (nk == 0) {
+        for (int g = tid; g < G; g += blockDim.x) part_lse[prow * Hq + hk * G + g] = -INFINITY;
+        return;
+    }
+    // stage K and V rows of this split, and the G query rows (pre-scaled)
+    constexpr int PIECES = D / 8;  // 16-byte pieces per row
+    const __nv_bfloat16 *kbase = k + ((static_cast<long long>(b) * T + k0) * Hkv + hk) * D;
+    const __nv_bfloat16 *vbase = v + ((static_cast<long long>(b) * T + k0) * Hkv + hk) * D;
+    for (int e = tid; e < nk * PIECES; e += blockDim.x) {
+        const int r = e / PIECES, c = e % PIECES;
+        const long long goff = static_cast<long long>(r) * Hkv * D + c * 8;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                         static_cast<uint32_t>(__cvta_generic_to_shared(Ks + r * KSTR + c * 8))),
+                     "l"(kbase + goff)
+                     : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                         static_cast<uint32_t>(__cvta_generic_to_shared(Vs + r * D + c * 8))),
+                     "l"(vbase + goff)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const __nv_bfloat16 *qrow = q + (static_cast<long long>(b) * Hq + hk * G) * D;
+    for (int e = tid; e < G * D; e += blockDim.x) qs[e] = __bfloat162float(qrow[e]) * scale_log2;
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+
+    // scores (log2 domain): ps[g][key]
+    for (int e = tid; e < G * KS; e += blockDim.x) {
+        const int g = e / KS, key = e % KS;
+        float acc = -INFINITY;
+        if (key < nk) {
+            acc = 0.f;
+            const uint4 *kr = reinterpret_cast<const uint4 *>(Ks + key * KSTR);
+            const float *qg = qs + g * D;
+#pragma unroll 4
+            for (int c = 0; c < PIECES; ++c) {
+                float kf[8];
+                bf16x8_to_f32(kr[c], kf);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc = fmaf(qg[c * 8 + u], kf[u], acc);
+            }
+        }
+        ps[e] = acc;
+    }
+    __syncthreads();
+    // per-head max and sum (one warp per head)
+    const int warp = tid / 32, lane = tid % 32;
+    for (int g = warp; g < G; g += blockDim.x / 32) {
+        float mx = -INFINITY;
+        for (int key = lane; key < nk; key += 32) mx = fmaxf(mx, ps[g * KS + key]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        float sum = 0.f;
+        for (int key = lane; key < KS; key += 32) {
+            const float pv = key < nk ? exp2f(ps[g * KS + key] - mx) : 0.f;
+            ps[g * KS + key] = pv;
+            sum += pv;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        if (lane == 0) {
+            ms[g] = mx;
+            ls[g] = sum;
+        }
+    }
+    __syncthreads();
+    // out[g][c] = sum_key p[g][key] * V[key][c] / l[g]
+    for (int e = tid; e < G * D; e += blockDim.x) {
+        const int g = e / D, c = e % D;
+        float acc = 0.f;
+        const float *pg = ps + g * KS;
+        for (int key = 0; key < nk; ++key) acc = fmaf(pg[key], __bfloat162float(Vs[key * D + c]), acc);
+        part_o[(prow * Hq + hk * G + g) * D + c] = acc / ls[g];
+    }
+    for (int g = tid; g < G; g += blockDim.x)
+        part_lse[prow * Hq + hk * G + g] = (ms[g] + log2f(ls[g])) * kLn2;
+}
+
+// ------------------------------------------------------------------------
+// Log-sum-exp combine: one warp per (query row, head); P = K*S partials,
+// slot s valid when ids[row][s] >= 0 and the partial's lse is finite.
+// ------------------------------------------------------------------------
+template <typename PT, int D>
+__global__ void __launch_bounds__(256) lse_combine_kernel(
+    const PT *__restrict__ part_o, const float *__restrict__ part_lse,
+    const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out,
+    long long rows, int Hq, int K, int S) {
+    constexpr int PER = D / 32;  // elements per lane
+    const long long w = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (w >= rows * Hq) return;
+    const long long row = w / Hq;
+    const int h = static_cast<int>(w % Hq);
+    float mx = -INFINITY;
+    for (int s = 0; s < K; ++s) {
+        if (ids[row * K + s] < 0) continue;
+        for (int p = 0; p < S; ++p) mx = fmaxf(mx, part_lse[((row * K + s) * S + p) * Hq + h]);
+    }
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+    float L = -INFINITY;
+    if (mx != -INFINITY) {
+        float sum = 0.f;
+        for (int s = 0; s < K; ++s) {
+            if (ids[row * K + s] < 0) continue;
+            for (int p = 0; p < S; ++p) {
+                const float l = part_lse[((row * K + s) * S + p) * Hq + h];
+                if (l != -INFINITY) sum += exp2f((l - mx) * kLog2e);
+            }
+        }
+        L = mx + log2f(sum) * kLn2;
+        for (int s = 0; s < K; ++s) {
+            if (ids[row * K + s] < 0) continue;
+            for (int p = 0; p < S; ++p) {
+                const long long pr = (row * K + s) * S + p;
+                const float l = part_lse[pr * Hq + h];
+                if (l == -INFINITY) continue;
+                const float wgt = exp2f((l - L) * kLog2e);
+                const PT *src = part_o + (pr * Hq + h) * D + lane * PER;
+#pragma unroll
+                for (int e = 0; e < PER; ++e) acc[e] = fmaf(wgt, static_cast<float>(src[e]), acc[e]);
+            }
+        }
+    }
+    float *dst = out + (row * Hq + h) * D + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) dst[e] = acc[e];
+    if (lane == 0) lse_out[row * Hq + h] = L;
+}
+
+// ------------------------------------------------------------------------
+// Inversion.  Chunks of kInvRows query rows; warp w of a chunk owns rows
+// [32w, 32w+32).  Per-warp histograms live in shared memory [4][N].
+// ------------------------------------------------------------------------
+__device__ __forceinline__ void warp_histogram(const int32_t *__restrict__ ids, int *hist_w,
+                                               int b, int n_q, int K, int N, int row0,
+                                               int *status) {
+    const int lane = threadIdx.x % 32;
+    const int i = row0 + lane;
+    if (i < n_q) {
+        const int32_t *r = ids + (static_cast<long long>(b) * n_q + i) * K;
+        for (int s = 0; s < K; ++s) {
+            const int j = r[s];
+            if (j >= 0 && j < N)
+                atomicAdd(hist_w + j, 1);
+            else if (j != -1 && status)
+                atomicOr(status, kDevBadIds);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(128) inv_count_kernel(const int32_t *__restrict__ ids,
+                                                         int *__restrict__ chunk_counts, int n_q,
+                                                         int K, int N, int n_chunks,
+                                                         int *__restrict__ status) {
+    extern __shared__ int hist[];  // [4][N]
+    const int chunk = blockIdx.x, b = blockIdx.y;
+    for (int e = threadIdx.x; e < 4 * N; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int w = threadIdx.x / 32;
+    warp_histogram(ids, hist + w * N, b, n_q, K, N, chunk * kInvRows + 32 * w, status);
+    __syncthreads();
+    int *dst = chunk_counts + (static_cast<long long>(b) * n_chunks + chunk) * N;
+    for (int j = threadIdx.x; j < N; j += blockDim.x)
+        dst[j] = hist[j] + hist[N + j] + hist[2 * N + j] + hist[3 * N + j];
+}
+
+// Exclusive scan of one (b, j) column over the chunks, in place; total out.
+__global__ void __launch_bounds__(256) inv_colscan_kernel(int *__restrict__ chunk_counts,
+                                                           int *__restrict__ pair_totals, int N,
+                                                           int n_chunks) {
+    const int j = blockIdx.x, b = blockIdx.y;
+    int *col = chunk_counts + static_cast<long long>(b) * n_chunks * N + j;
+    __shared__ int warp_sums[8];
+    const int per = (n_chunks + blockDim.x - 1) / blockDim.x;
+    const int c0 = threadIdx.x * per;
+    int local = 0;
+    for (int c = c0; c < min(c0 + per, n_chunks); ++c) local += col[static_cast<long long>(c) * N];
+    // block exclusive scan of `local`
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int warp_off = 0;
+    for (int x = 0; x < warp; ++x) warp_off += warp_sums[x];
+    int run = warp_off + incl - local;
+    for (int c = c0; c < min(c0 + per, n_chunks); ++c) {
+        const long long o = static_cast<long long>(c) * N;
+        const int v = col[o];
+        col[o] = run;
+        run += v;
+    }
+    if (threadIdx.x == blockDim.x - 1) {
+        int tot = 0;
+        for (int x = 0; x < static_cast<int>(blockDim.x / 32); ++x) tot += warp_sums[x];
+        pair_totals[static_cast<long long>(b) * N + j] = tot;
+    }
+}
+
+// Single-CTA exclusive scans: row_ptr over pair totals; item_ptr over
+// ceil(total / rows_per_item) (when items != nullptr); counters[0] = items,
+// counters[1] = 0 (work cursor of the attention kernel).
+__global__ void __launch_bounds__(1024) inv_rowptr_kernel(const int *__restrict__ pair_totals,
+                                                           int *__restrict__ row_ptr,
+                                                           int *__restrict__ item_ptr,
+                                                           int *__restrict__ counters, int n_pairs,
+                                                           int rows_per_item) {
+    __shared__ int ws_a[32], ws_b[32];
+    const int per = (n_pairs + blockDim.x - 1) / blockDim.x;
+    const int p0 = threadIdx.x * per;
+    int la = 0, lb = 0;
+    for (int p = p0; p < min(p0 + per, n_pairs); ++p) {
+        la += pair_totals[p];
+        if (item_ptr) lb += (pair_totals[p] + rows_per_item - 1) / rows_per_item;
+    }
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    int ia = la, ib = lb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xFFFFFFFFu, ia, o);
+        const int yb = __shfl_up_sync(0xFFFFFFFFu, ib, o);
+        if (lane >= o) {
+            ia += ya;
+            ib += yb;
+        }
+    }
+    if (lane == 31) {
+        ws_a[warp] = ia;
+        ws_b[warp] = ib;
+    }
+    __syncthreads();
+    int oa = 0, ob = 0;
+    for (int x = 0; x < warp; ++x) {
+        oa += ws_a[x];
+        ob += ws_b[x];
+    }
+    int ra = oa + ia - la, rb = ob + ib - lb;
+    for (int p = p0; p < min(p0 + per, n_pairs); ++p) {
+        row_ptr[p] = ra;
+        ra += pair_totals[p];
+        if (item_ptr) {
+            item_ptr[p] = rb;
+            rb += (pair_totals[p] + rows_per_item - 1) / rows_per_item;
+        }
+    }
+    if (threadIdx.x == blockDim.x - 1) {
+        int ta = 0, tb = 0;
+        for (int x = 0; x < static_cast<int>(blockDim.x / 32); ++x) {
+            ta += ws_a[x];
+            tb += ws_b[x];
+        }
+        row_ptr[n_pairs] = ta;
+        if (item_ptr) {
+            item_ptr[n_pairs] = tb;
+            counters[0] = tb;
+            counters[1] = 0;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(128) inv_scatter_kernel(
+    const int32_t *__restrict__ ids, const int *__restrict__ chunk_prefix,
+    const int *__restrict__ row_ptr, int32_t *__restrict__ entries, int n_q, int K, int N,
+    int n_chunks, int *__restrict__ status) {
+    extern __shared__ int hist[];  // [4][N] counts, then cursors
+    const int chunk = blockIdx.x, b = blockIdx.y;
+    for (int e = threadIdx.x; e < 4 * N; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
+    // bad ids were already reported by the count pass
+    warp_histogram(ids, hist + w * N, b, n_q, K, N, chunk * kInvRows + 32 * w, nullptr);
+    (void)status;
+    __syncthreads();
+    const int *pre = chunk_prefix + (static_cast<long long>(b) * n_chunks + chunk) * N;
+    for (int j = threadIdx.x; j < N; j += blockDim.x) {
+        int base = row_ptr[static_cast<long long>(b) * N + j] + pre[j];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int c = hist[x * N + j];
+            hist[x * N + j] = base;
+            base += c;
+        }
+    }
+    __syncthreads();
+    int *cursor = hist + w * N;
+    const int row0 = chunk * kInvRows + 32 * w;
+    for (int r = 0; r < 32; ++r) {
+        const int i = row0 + r;
+        if (i >= n_q) break;
+        const long long row = static_cast<long long>(b) * n_q + i;
+        if (lane < K) {
+            const int j = ids[row * K + lane];
+            if (j >= 0 && j < N) {
+                const int pos = atomicAdd(cursor + j, 1);
+                entries[pos] = static_cast<int32_t>(row * K + lane);
+            }
+        }
+        __syncwarp();
+    }
+}
+
+__global__ void __launch_bounds__(256) attn_items_kernel(const int *__restrict__ pair_totals,
+                                                          const int *__restrict__ item_ptr,
+                                                          AttnItem *__restrict__ items,
+                                                          int n_pairs, int rows_per_item) {
+    const int p = blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= n_pairs) return;
+    const int tot = pair_totals[p];
+    int o = item_ptr[p];
+    for (int s = 0; s < tot; s += rows_per_item) {
+        AttnItem it;
+        it.pair = p;
+        it.start = s;
+        it.count = min(rows_per_item, tot - s);
+        it.pad = 0;
+        items[o++] = it;
+    }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_decode_index(const Shape &sh, const void *q_idx, const void *k_idx,
+                                int32_t *ids, float *block_scores, int num_sms,
+                                cudaStream_t st) {
+    const int own = (sh.T - 1) / sh.block;
+    if (own > 0) {
+        const long long work = static_cast<long long>(sh.Bt) * own;
+        long long blocks = (work + 7) / 8;
+        const long long cap = static_cast<long long>(num_sms) * 8;
+        if (blocks > cap) blocks = cap;
+        const auto *qi = static_cast<const __nv_bfloat16 *>(q_idx);
+        const auto *ki = static_cast<const __nv_bfloat16 *>(k_idx);
+        if (sh.d_idx == 128)
+            decode_index_scan_kernel<128><<<static_cast<int>(blocks), 256, 0, st>>>(
+                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N);
+        else
+            decode_index_scan_kernel<64><<<static_cast<int>(blocks), 256, 0, st>>>(
+                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N);
+    }
+    if (sh.K <= 8)
+        decode_select_kernel<7><<<sh.Bt, 32, 0, st>>>(block_scores, ids, sh.N, own, sh.K);
+    else if (sh.K <= 16)
+        decode_select_kernel<15><<<sh.Bt, 32, 0, st>>>(block_scores, ids, sh.N, own, sh.K);
+    else
+        decode_select_kernel<31><<<sh.Bt, 32, 0, st>>>(block_scores, ids, sh.N, own, sh.K);
+    return cudaGetLastError();
+}
+
+size_t decode_attn_smem_bytes(const Shape &sh) {
+    const int G = sh.G;
+    size_t f = static_cast<size_t>(G) * sh.d + static_cast<size_t>(G) * kDecodeKeys + 2 * G;
+    size_t bytes = align_up(f * 4, 16);
+    bytes += static_cast<size_t>(kDecodeKeys) * (sh.d + 8) * 2 + static_cast<size_t>(kDecodeKeys) * sh.d * 2;
+    return bytes;
+}
+
+cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, const void *v,
+                               const int32_t *ids, float *part_o, float *part_lse, int S,
+                               int *status, cudaStream_t st) {
+    const long long grid = static_cast<long long>(sh.Bt) * sh.Hkv * sh.K * S;
+    const size_t smem = decode_attn_smem_bytes(sh);
+    const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(sh.d));
+    const auto *qb = static_cast<const __nv_bfloat16 *>(q);
+    const auto *kb = static_cast<const __nv_bfloat16 *>(k);
+    const auto *vb = static_cast<const __nv_bfloat16 *>(v);
+    if (sh.d == 128) {
+        cudaFuncSetAttribute(decode_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+        decode_attn_kernel<128><<<static_cast<unsigned>(grid), 128, smem, st>>>(
+            qb, kb, vb, ids, part_o, part_lse, sh.T, sh.Hq, sh.Hkv, sh.block, sh.K, S, sh.N,
+            scale_log2, status);
+    } else {
+        cudaFuncSetAttribute(decode_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+        decode_attn_kernel<64><<<static_cast<unsigned>(grid), 128, smem, st>>>(
+            qb, kb, vb, ids, part_o, part_lse, sh.T, sh.Hq, sh.Hkv, sh.block, sh.K, S, sh.N,
+            scale_log2, status);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
+                           const float *part_lse, const int32_t *ids, float *out, float *lse,
+                           int S, cudaStream_t st) {
+    const long long rows = static_cast<long long>(sh.Bt) * sh.n_q;
+    const long long warps = rows * sh.Hq;
+    const long long blocks = (warps + 7) / 8;
+    if (part_bf16) {
+        const auto *po = static_cast<const __nv_bfloat16 *>(part_o);
+        if (sh.d == 128)
+            lse_combine_kernel<__nv_bfloat16, 128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+                po, part_lse, ids, out, lse, rows, sh.Hq, sh.K, S);
+        else
+            lse_combine_kernel<__nv_bfloat16, 64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+                po, part_lse, ids, out, lse, rows, sh.Hq, sh.K, S);
+    } else {
+        const auto *po = static_cast<const float *>(part_o);
+        if (sh.d == 128)
+            lse_combine_kernel<float, 128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+                po, part_lse, ids, out, lse, rows, sh.Hq, sh.K, S);
+        else
+            lse_combine_kernel<float, 64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+                po, part_lse, ids, out, lse, rows, sh.Hq, sh.K, S);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts,
+                          int *pair_totals, int32_t *row_ptr, int32_t *entries, int *item_ptr,
+                          AttnItem *items, int *counters, int rows_per_item, int n_chunks,
+                          int *status, cudaStream_t st) {
+    const size_t hist_bytes = static_cast<size_t>(4) * sh.N * sizeof(int);
+    cudaFuncSetAttribute(inv_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(hist_bytes));
+    cudaFuncSetAttribute(inv_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(hist_bytes));
+    const dim3 cgrid(n_chunks, sh.Bt);
+    inv_count_kernel<<<cgrid, 128, hist_bytes, st>>>(ids, chunk_counts, sh.n_q, sh.K, sh.N,
+                                                      n_chunks, status);
+    inv_colscan_kernel<<<dim3(sh.N, sh.Bt), 256, 0, st>>>(chunk_counts, pair_totals, sh.N,
+                                                           n_chunks);
+    const int n_pairs = sh.Bt * sh.N;
+    inv_rowptr_kernel<<<1, 1024, 0, st>>>(pair_totals, row_ptr, item_ptr, counters, n_pairs,
+                                          rows_per_item);
+    inv_scatter_kernel<<<cgrid, 128, hist_bytes, st>>>(ids, chunk_counts, row_ptr, entries,
+                                                        sh.n_q, sh.K, sh.N, n_chunks, status);
+    if (items)
+        attn_items_kernel<<<(n_pairs + 255) / 256, 256, 0, st>>>(pair_totals, item_ptr, items,
+                                                                  n_pairs, rows_per_item);
+    return cudaGetLastError();
+}
+
+}  // namespace msa

@@ -1,0 +1,771 @@
+// kernels_tc.cu -- tcgen05 (5th-generation tensor core) kernels of the MSA
+// hot path on sm_100a:
+//   * prefill_index_kernel: index branch for many queries.  S = q_idx k_idx^T
+//     tiles (128 queries x 128 keys) accumulate in tensor memory; the
+//     epilogue warps max-pool each key block and keep a register top-K per
+//     query row, so the n_q x T score matrix never exists.
+//   * prefill_attn_kernel: sparse branch, KV-block-outer.  Each work item is
+//     one (sequence, block, kv head) hit list (or a slice of it): the block's
+//     K and V are TMA-loaded into shared memory once, the hit queries' G heads
+//     are gathered as 128-row tiles, S = QK^T and O = PV run on tcgen05 with
+//     the online softmax in between, and a normalised partial (O, lse) per
+//     (query, slot, head) goes to the workspace for the log-sum-exp combine.
+//   * selftest_umma_kernel: one 128 x N GEMM through the same TMA /
+//     descriptor / MMA / TMEM code, for validating the building blocks.
+//
+// Method: "MiniMax M3模型算力成本大幅降低原因深度解析" (index branch: single-head
+// key, block max-pool, top-K; sparse branch: GQA on the kept blocks, raw KV)
+// and "MiniMax M3 深度实战", section 2.2 (KV outer gather Q, each KV block read
+// once) and section 2.3 (local block always kept; softmax(QK^T/sqrt(d))V).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cstdint>
+
+#include "kernels.h"
+#include "msa_common.cuh"
+#include "ptx_sm100.cuh"
+
+namespace msa {
+
+namespace {
+
+constexpr float kLn2f = 0.6931471805599453f;
+constexpr uint32_t kRegionBytes = 16384;  // 128 rows x 128 B (64 bf16) swizzled region
+
+__device__ __forceinline__ unsigned char *align1024(unsigned char *p) {
+    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+}
+
+// Bounded wait that ignores the abort flag: used only to drain copies that
+// are still in flight when a kernel unwinds after an abort.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs / 4) break;
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// ===========================================================================
+// Self-test GEMM: C[128][N] = A[128][Kd] . B, one CTA of 128 threads.
+// ===========================================================================
+__global__ void __launch_bounds__(128, 1) selftest_umma_kernel(
+    const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+    float *__restrict__ C, int N, int Kd, int b_mn_major, int *status) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = align1024(smem_raw);
+    unsigned char *a_s = base;                                  // Kd/64 regions x 16 KB
+    unsigned char *b_s = a_s + (Kd / 64) * kRegionBytes;        // Kd*N*2 bytes
+    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(b_s + static_cast<size_t>(Kd) * N * 2);
+    uint64_t *bar_mma = bar_ld + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid / 32;
+    const uint32_t ncols = N <= 64 ? 64u : (N <= 128 ? 128u : 256u);
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_mma, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, ncols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (tid == 0) {
+        const uint32_t bytes = static_cast<uint32_t>(128 * Kd * 2 + Kd * N * 2);
+        mbar_arrive_expect_tx(bar_ld, bytes);
+        for (int r = 0; r < Kd / 64; ++r) tma_load_2d(a_s + r * kRegionBytes, &tm_a, bar_ld, r * 64, 0);
+        if (b_mn_major) {
+            // B [Kd][N]: N/64 regions, each Kd rows x 128 B
+            for (int r = 0; r < N / 64; ++r)
+                tma_load_2d(b_s + static_cast<size_t>(r) * Kd * 128, &tm_b, bar_ld, r * 64, 0);
+        } else {
+            // B [N][Kd]: Kd/64 regions, each N rows x 128 B
+            for (int r = 0; r < Kd / 64; ++r)
+                tma_load_2d(b_s + static_cast<size_t>(r) * N * 128, &tm_b, bar_ld, r * 64, 0);
+        }
+    }
+    bool ok = mbar_wait(bar_ld, 0, abort_flag, status);
+    if (ok && tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16_f32(128, N, b_mn_major != 0);
+        for (int kk = 0; kk < Kd / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(smem_addr(a_s + (kk / 4) * kRegionBytes + (kk % 4) * 32), 16, 1024);
+            uint64_t bd;
+            if (b_mn_major)
+                bd = sdesc_sw128(smem_addr(b_s + kk * 16 * 128), static_cast<uint32_t>(Kd) * 128, 1024);
+            else
+                bd = sdesc_sw128(smem_addr(b_s + static_cast<size_t>(kk / 4) * N * 128 + (kk % 4) * 32), 16, 1024);
+            umma_bf16(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_mma);
+    }
+    ok = ok && mbar_wait(bar_mma, 0, abort_flag, status);
+    __syncwarp();
+    tc_fence_after();
+    if (__all_sync(0xFFFFFFFFu, ok)) {
+        const int row = warp * 32 + (tid % 32);
+        for (int c = 0; c < N / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c * 32, v);
+            tmem_wait_ld();
+            for (int e = 0; e < 32; ++e) C[static_cast<size_t>(row) * N + c * 32 + e] = __uint_as_float(v[e]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+// ===========================================================================
+// Prefill index kernel.
+//   warp 0: TMA producer (q tile once per item, 128-key k tiles through a
+//           4-stage ring), warp 1: MMA issuer (TMEM owner), warps 2-5:
+//           epilogue (row = 32*(warp%4) + lane; block max-pool + top-K).
+// Work item = (sequence b, 128-query tile qt); items ordered by decreasing
+// cost and dealt to CTAs in a snake order.
+// ===========================================================================
+struct IndexParams {
+    int32_t *ids;
+    int *status;
+    int Bt, n_q, T, block, K, n_qt, n_items;
+};
+
+constexpr int kIdxStages = 4;
+
+__device__ __forceinline__ int snake_item(int it, int cta, int ncta) {
+    return (it & 1) ? it * ncta + (ncta - 1 - cta) : it * ncta + cta;
+}
+
+template <int CAP>
+__device__ __forceinline__ void topk_insert(float (&ts)[CAP], int (&tj)[CAP], float s, int j) {
+    if (!(s > ts[CAP - 1])) return;
+    bool ins = false;
+#pragma unroll
+    for (int p = 0; p < CAP; ++p) {
+        const bool take = ins || s > ts[p];
+        if (take) {
+            const float fs = ts[p];
+            const int ij = tj[p];
+            ts[p] = s;
+            tj[p] = j;
+            s = fs;
+            j = ij;
+            ins = true;
+        }
+    }
+}
+
+template <int D_IDX, int CAP>
+__global__ void __launch_bounds__(192, 1) prefill_index_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    IndexParams p) {
+    constexpr int NREG = D_IDX / 64;
+    constexpr uint32_t TILE = NREG * kRegionBytes;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = align1024(smem_raw);
+    unsigned char *q_s = base;
+    unsigned char *k_s = base + TILE;  // kIdxStages tiles
+    uint64_t *bars = reinterpret_cast<uint64_t *>(k_s + kIdxStages * TILE);
+    uint64_t *kfull = bars;
+    uint64_t *kempty = bars + kIdxStages;
+    uint64_t *qfull = bars + 2 * kIdxStages;
+    uint64_t *qempty = qfull + 1;
+    uint64_t *tfull = qfull + 2;   // [2]
+    uint64_t *tempty = qfull + 4;  // [2]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qfull + 6);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    if (tid == 0) {
+        for (int s = 0; s < kIdxStages; ++s) {
+            mbar_init(kfull + s, 1);
+            mbar_init(kempty + s, 1);
+        }
+        mbar_init(qfull, 1);
+        mbar_init(qempty, 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull + a, 1);
+            mbar_init(tempty + a, 128);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int B = p.block;
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            uint32_t n = 0;
+            bool ok = true;
+            int armed[kIdxStages];
+            for (int s = 0; s < kIdxStages; ++s) armed[s] = -1;
+            for (int it = 0; ok; ++it) {
+                const int idx = snake_item(it, blockIdx.x, gridDim.x);
+                if (idx >= p.n_items) break;
+                const int qt = p.n_qt - 1 - idx / p.Bt, b = idx % p.Bt;
+                const int i_last = min(qt * 128 + 127, p.n_q - 1);
+                const int own_max = (p.T - p.n_q + i_last) / B;
+                const int n_sub = (own_max * B + 127) / 128;
+                if (!mbar_wait(qempty, (it & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+                mbar_arrive_expect_tx(qfull, TILE);
+                for (int r = 0; r < NREG; ++r)
+                    tma_load_2d(q_s + r * kRegionBytes, &tm_q, qfull, r * 64, b * p.n_q + qt * 128);
+                for (int s = 0; s < n_sub; ++s, ++n) {
+                    const uint32_t st = n % kIdxStages, rd = n / kIdxStages;
+                    if (!mbar_wait(kempty + st, (rd & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(kfull + st, TILE);
+                    armed[st] = static_cast<int>(rd & 1);
+                    for (int r = 0; r < NREG; ++r)
+                        tma_load_2d(k_s + st * TILE + r * kRegionBytes, &tm_k, kfull + st, r * 64,
+                                    b * p.T + s * 128);
+                }
+            }
+            if (*abort_flag) {  // drain this CTA's copies still in flight
+                for (int s = 0; s < kIdxStages; ++s)
+                    if (armed[s] >= 0) mbar_drain(kfull + s, static_cast<uint32_t>(armed[s]));
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, 128, false);
+            uint32_t n = 0, acc_n = 0;
+            bool ok = true;
+            for (int it = 0; ok; ++it) {
+                const int idx = snake_item(it, blockIdx.x, gridDim.x);
+                if (idx >= p.n_items) break;
+                const int qt = p.n_qt - 1 - idx / p.Bt;
+                const int i_last = min(qt * 128 + 127, p.n_q - 1);
+                const int own_max = (p.T - p.n_q + i_last) / B;
+                const int n_sub = (own_max * B + 127) / 128;
+                if (!mbar_wait(qfull, it & 1, abort_flag, p.status)) break;
+                for (int s = 0; s < n_sub; ++s, ++n, ++acc_n) {
+                    const uint32_t st = n % kIdxStages, rd = n / kIdxStages;
+                    const uint32_t acc = acc_n & 1, ar = acc_n >> 1;
+                    if (!mbar_wait(kfull + st, rd & 1, abort_flag, p.status)) { ok = false; break; }
+                    if (!mbar_wait(tempty + acc, (ar & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t qa = smem_addr(q_s), ka = smem_addr(k_s + st * TILE);
+#pragma unroll
+                    for (int kk = 0; kk < D_IDX / 16; ++kk) {
+                        const uint32_t off = (kk / 4) * kRegionBytes + (kk % 4) * 32;
+                        umma_bf16(tmem + acc * 128, sdesc_sw128(qa + off, 16, 1024),
+                                  sdesc_sw128(ka + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(kempty + st);
+                    umma_commit(tfull + acc);
+                }
+                umma_commit(qempty);
+            }
+        }
+    } else {
+        // epilogue warps 2..5
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        uint32_t acc_n = 0;
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int idx = snake_item(it, blockIdx.x, gridDim.x);
+            if (idx >= p.n_items) break;
+            const int qt = p.n_qt - 1 - idx / p.Bt, b = idx % p.Bt;
+            const int i_last = min(qt * 128 + 127, p.n_q - 1);
+            const int own_max = (p.T - p.n_q + i_last) / B;
+            const int n_sub = (own_max * B + 127) / 128;
+            const int i = qt * 128 + row;
+            const bool valid = i < p.n_q;
+            const int own = valid ? (p.T - p.n_q + i) / B : 0;
+            float ts[CAP];
+            int tj[CAP];
+#pragma unroll
+            for (int q = 0; q < CAP; ++q) {
+                ts[q] = -FLT_MAX;
+                tj[q] = 0x7FFFFFFF;
+            }
+            float bm = -FLT_MAX;
+            for (int s = 0; s < n_sub; ++s, ++acc_n) {
+                const uint32_t acc = acc_n & 1, ar = acc_n >> 1;
+                if (!mbar_wait(tfull + acc, ar & 1, abort_flag, p.status)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_addr + acc * 128 + c * 32, v);
+                    tmem_wait_ld();
+                    // block >= 32 and 32 | block: a 32-column chunk lies in one block
+                    float m = -FLT_MAX;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) m = fmaxf(m, __uint_as_float(v[e]));
+                    bm = fmaxf(bm, m);
+                    const int col_end = s * 128 + c * 32 + 32;
+                    if (col_end % B == 0) {
+                        const int j = col_end / B - 1;
+                        if (j < own) topk_insert<CAP>(ts, tj, bm, j);
+                        bm = -FLT_MAX;
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(tempty + acc);
+            }
+            if (!ok) break;
+            if (valid) {
+                const int m = min(p.K, own + 1) - 1;
+                int a[CAP + 1];
+#pragma unroll
+                for (int q = 0; q < CAP; ++q) a[q] = q < m ? tj[q] : 0x7FFFFFFF;
+                a[CAP] = own;
+                // odd-even transposition sort, ascending
+#pragma unroll
+                for (int r = 0; r < CAP + 1; ++r) {
+#pragma unroll
+                    for (int q = (r & 1); q + 1 < CAP + 1; q += 2) {
+                        const int lo = min(a[q], a[q + 1]), hi = max(a[q], a[q + 1]);
+                        a[q] = lo;
+                        a[q + 1] = hi;
+                    }
+                }
+                int32_t *dst = p.ids + (static_cast<long long>(b) * p.n_q + i) * p.K;
+#pragma unroll
+                for (int q = 0; q < CAP + 1; ++q)
+                    if (q < p.K) dst[q] = a[q] == 0x7FFFFFFF ? -1 : a[q];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// ===========================================================================
+// Prefill attention (KV-block-outer).
+// ===========================================================================
+struct AttnParams {
+    const __nv_bfloat16 *q;
+    const int32_t *row_ptr;
+    const int32_t *entries;
+    const AttnItem *items;
+    int *counters;  // [0] items per kv head, [1] work cursor
+    __nv_bfloat16 *part_o;
+    float *part_lse;
+    int *status;
+    int Bt, n_q, T, Hq, Hkv, G, block, K, N;
+    int NK;   // keys per sub-tile (min(block, 128))
+    int NS;   // sub-tiles per block
+    int TOK;  // tokens per 128-row chunk = 128 / G
+    float scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 1) prefill_attn_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    AttnParams p) {
+    constexpr int DREG = D / 64;                 // swizzled regions per Q row block
+    constexpr uint32_t QBYTES = DREG * kRegionBytes;
+    const int NK = p.NK;
+    const uint32_t kv_tile = static_cast<uint32_t>(NK) * 128u * DREG;  // one of K or V
+    const int KVST = p.NS > 1 ? 2 : 1;
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = align1024(smem_raw);
+    unsigned char *kv_s = base;                                   // KVST x (K tile, V tile)
+    unsigned char *q_s = kv_s + KVST * 2 * kv_tile;               // 2 x QBYTES
+    unsigned char *p_s = q_s + 2 * QBYTES;                        // NK/64 regions
+    unsigned char *tail = p_s + ((NK + 63) / 64) * kRegionBytes;
+    uint64_t *kvfull = reinterpret_cast<uint64_t *>(tail);        // [2]
+    uint64_t *bar_s = kvfull + 2;
+    uint64_t *bar_o = kvfull + 3;
+    int *tok_entry = reinterpret_cast<int *>(kvfull + 4);         // [2][128]
+    int *sh_item = tok_entry + 256;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sh_item + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid / 32;
+    if (tid == 0) {
+        mbar_init(kvfull, 1);
+        mbar_init(kvfull + 1, 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_s = tmem;        // S: columns [0, NK)
+    const uint32_t tmem_o = tmem + 128;  // O: columns [128, 128 + D)
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+
+    const int n_items = p.counters[0];
+    const int total = n_items * p.Hkv;
+    const int G = p.G, TOK = p.TOK, K = p.K;
+    const uint32_t idesc_s = idesc_bf16_f32(128, NK, false);
+    const uint32_t idesc_o = idesc_bf16_f32(128, D, true);
+    const int row = tid;  // M row of this thread (TMEM lane)
+    const int tok = row / G, g = row % G;
+
+    uint32_t kv_issue = 0, kv_use = 0, s_n = 0, o_n = 0;
+    int armed_parity[2] = {-1, -1};
+    bool aborted = false;
+
+    // Issue the K/V loads of sub-tile kt of block (b, j), kv head hk.
+    auto issue_kv = [&](int b, int j, int hk, int kt) {
+        const uint32_t st = kv_issue % KVST;
+        unsigned char *kd = kv_s + st * 2 * kv_tile;
+        unsigned char *vd = kd + kv_tile;
+        mbar_arrive_expect_tx(kvfull + st, 2 * kv_tile);
+        armed_parity[st] = static_cast<int>((kv_issue / KVST) & 1);
+        const int z = b * p.T + j * p.block + kt * NK;
+        for (int r = 0; r < DREG; ++r) {
+            tma_load_3d(kd + r * NK * 128, &tm_k, kvfull + st, r * 64, hk, z);
+            tma_load_3d(vd + r * NK * 128, &tm_v, kvfull + st, r * 64, hk, z);
+        }
+        ++kv_issue;
+    };
+
+    // Gather the G heads of the chunk's tokens into Q buffer qb (cp.async).
+    auto gather_q = [&](int qb, int hk, int b, int list_base, int chunk, int ntok_item) {
+        unsigned char *dst_base = q_s + qb * QBYTES;
+        const int tok0 = chunk * TOK;
+        if (tid < TOK) {
+            int e = -1;
+            if (tok0 + tid < ntok_item) {
+                e = p.entries[list_base + tok0 + tid];
+                const long long qrow = e / K;
+                if (e < 0 || qrow >= static_cast<long long>(p.Bt) * p.n_q || qrow / p.n_q != b) {
+                    atomicOr(p.status, kDevBadIds);
+                    e = -1;
+                }
+            }
+            tok_entry[qb * 128 + tid] = e;
+        }
+        constexpr int PPR = D / 8;  // 16-byte pieces per row
+        for (int pc = tid; pc < 128 * PPR; pc += 128) {
+            const int r = pc / PPR, cc = pc % PPR;
+            const int tk = r / G, gg = r % G;
+            int e = -1;
+            if (tok0 + tk < ntok_item) e = p.entries[list_base + tok0 + tk];
+            const long long qrow = e / K;
+            const bool ok = e >= 0 && qrow < static_cast<long long>(p.Bt) * p.n_q && qrow / p.n_q == b;
+            const __nv_bfloat16 *src =
+                ok ? p.q + ((qrow * p.Hq + hk * G + gg) * D + cc * 8) : p.q;
+            unsigned char *dst = dst_base + (cc / 8) * kRegionBytes + sw128_offset(r, cc % 8);
+            cp_async_16(dst, src, ok ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+
+    while (true) {
+        if (tid == 0) *sh_item = atomicAdd(p.counters + 1, 1);
+        __syncthreads();
+        const int w = *sh_item;
+        if (w >= total) break;
+        const int hk = w / n_items;
+        const AttnItem item = p.items[w % n_items];
+        const int b = item.pair / p.N, j = item.pair % p.N;
+        const int list_base = p.row_ptr[item.pair] + item.start;
+        const int ntok = item.count;
+        const int n_chunks = (ntok + TOK - 1) / TOK;
+        const int n_steps = n_chunks * p.NS;
+
+        if (tid == 0) issue_kv(b, j, hk, 0);
+        gather_q(0, hk, b, list_base, 0, ntok);
+
+        float m_run = -INFINITY, l_run = 0.f;
+        for (int step = 0; step < n_steps; ++step) {
+            const int c = step / p.NS, kt = step % p.NS;
+            const int qb = c & 1;
+            if (kt == 0) cp_async_wait_all();
+            fence_proxy_async_smem();
+            __syncthreads();
+            // wait for this step's K/V tile
+            const uint32_t st = kv_use % KVST;
+            bool ok = true;
+            if (p.NS > 1 || c == 0) {
+                ok = mbar_wait(kvfull + st, (kv_use / KVST) & 1, abort_flag, p.status);
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+                ++kv_use;
+                armed_parity[st] = -1;
+            }
+            unsigned char *kd = kv_s + st * 2 * kv_tile;
+            unsigned char *vd = kd + kv_tile;
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t qa = smem_addr(q_s + qb * QBYTES), ka = smem_addr(kd);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    umma_bf16(tmem_s,
+                              sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
+                              sdesc_sw128(ka + (kk / 4) * NK * 128 + (kk % 4) * 32, 16, 1024),
+                              idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bar_s);
+                // prefetch the next sub-tile of this block (streamed K/V)
+                if (p.NS > 1 && step + 1 < n_steps) issue_kv(b, j, hk, (step + 1) % p.NS);
+            }
+            if (kt == 0 && c + 1 < n_chunks) gather_q(qb ^ 1, hk, b, list_base, c + 1, ntok);
+            ok = mbar_wait(bar_s, s_n & 1, abort_flag, p.status);
+            ++s_n;
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            tc_fence_after();
+
+            // ---- softmax for row `row`
+            const int e = tok_entry[qb * 128 + tok];
+            const bool valid = e >= 0;
+            const long long qrow = valid ? e / K : 0;
+            const int t = p.T - p.n_q + static_cast<int>(qrow % p.n_q);
+            const int kbase = j * p.block + kt * NK;
+            const int lim = valid ? t - kbase : -1;  // valid columns: col <= lim
+            float mt = -INFINITY;
+            for (int cc = 0; cc < NK / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(tmem_s + lane_addr + cc * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x)
+                    if (cc * 32 + x <= lim) mt = fmaxf(mt, __uint_as_float(v[x]));
+            }
+            mt *= p.scale_log2;
+            if (kt == 0) {
+                m_run = mt;
+                l_run = 0.f;
+            } else {
+                float alpha = 1.f;
+                bool need = false;
+                if (mt > m_run + 8.f) {
+                    alpha = exp2f(m_run - mt);
+                    m_run = mt;
+                    l_run *= alpha;
+                    need = true;
+                }
+                if (__any_sync(0xFFFFFFFFu, need)) {
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem_o + lane_addr + cc * 32, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
+                        tmem_st32(tmem_o + lane_addr + cc * 32, v);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            unsigned char *prow_base = p_s;
+            for (int cc = 0; cc < NK / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(tmem_s + lane_addr + cc * 32, v);
+                tmem_wait_ld();
+                float pv[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    const bool in = cc * 32 + x <= lim;
+                    pv[x] = in ? exp2f(__uint_as_float(v[x]) * p.scale_log2 - m_run) : 0.f;
+                    l_run += pv[x];
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int col = cc * 32 + q4 * 8;  // first key of this 16-byte piece
+                    uint4 u;
+                    u.x = pack_bf16x2(pv[q4 * 8 + 0], pv[q4 * 8 + 1]);
+                    u.y = pack_bf16x2(pv[q4 * 8 + 2], pv[q4 * 8 + 3]);
+                    u.z = pack_bf16x2(pv[q4 * 8 + 4], pv[q4 * 8 + 5]);
+                    u.w = pack_bf16x2(pv[q4 * 8 + 6], pv[q4 * 8 + 7]);
+                    *reinterpret_cast<uint4 *>(prow_base + (col / 64) * kRegionBytes +
+                                               sw128_offset(row, (col % 64) / 8)) = u;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t pa = smem_addr(p_s), va = smem_addr(vd);
+                for (int kk = 0; kk < NK / 16; ++kk) {
+                    umma_bf16(tmem_o,
+                              sdesc_sw128(pa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
+                              sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
+                              idesc_o, (kt > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bar_o);
+            }
+            ok = mbar_wait(bar_o, o_n & 1, abort_flag, p.status);
+            ++o_n;
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            tc_fence_after();
+
+            if (kt == p.NS - 1) {
+                // ---- epilogue: normalised partial and its lse
+                const int slot = valid ? static_cast<int>(e % K) : 0;
+                const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+                __nv_bfloat16 *dst =
+                    p.part_o + ((qrow * K + slot) * p.Hq + static_cast<long long>(hk) * G + g) * D;
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem_o + lane_addr + cc * 32, v);
+                    tmem_wait_ld();
+                    if (valid) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 u;
+                            u.x = pack_bf16x2(__uint_as_float(v[q4 * 8 + 0]) * inv_l, __uint_as_float(v[q4 * 8 + 1]) * inv_l);
+                            u.y = pack_bf16x2(__uint_as_float(v[q4 * 8 + 2]) * inv_l, __uint_as_float(v[q4 * 8 + 3]) * inv_l);
+                            u.z = pack_bf16x2(__uint_as_float(v[q4 * 8 + 4]) * inv_l, __uint_as_float(v[q4 * 8 + 5]) * inv_l);
+                            u.w = pack_bf16x2(__uint_as_float(v[q4 * 8 + 6]) * inv_l, __uint_as_float(v[q4 * 8 + 7]) * inv_l);
+                            *reinterpret_cast<uint4 *>(dst + cc * 32 + q4 * 8) = u;
+                        }
+                    }
+                }
+                if (valid)
+                    p.part_lse[(qrow * K + slot) * p.Hq + static_cast<long long>(hk) * G + g] =
+                        l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
+                m_run = -INFINITY;
+                l_run = 0.f;
+            }
+            tc_fence_before();
+        }
+        if (aborted) break;
+    }
+    __syncthreads();
+    if (aborted && tid == 0) {
+        for (int s = 0; s < 2; ++s)
+            if (armed_parity[s] >= 0) mbar_drain(kvfull + s, static_cast<uint32_t>(armed_parity[s]));
+    }
+    cp_async_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+size_t selftest_smem_bytes(int N, int Kd) {
+    return 1024 + static_cast<size_t>(Kd / 64) * kRegionBytes + static_cast<size_t>(Kd) * N * 2 + 64;
+}
+
+cudaError_t launch_selftest_umma(const CUtensorMap &tm_a, const CUtensorMap &tm_b, float *C,
+                                 int N, int Kd, int b_mn_major, int *status, cudaStream_t st) {
+    const size_t smem = selftest_smem_bytes(N, Kd);
+    cudaFuncSetAttribute(selftest_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    selftest_umma_kernel<<<1, 128, smem, st>>>(tm_a, tm_b, C, N, Kd, b_mn_major, status);
+    return cudaGetLastError();
+}
+
+size_t prefill_index_smem_bytes(int d_idx) {
+    return 1024 + static_cast<size_t>(1 + kIdxStages) * (d_idx / 64) * kRegionBytes + 256;
+}
+
+template <int D_IDX, int CAP>
+static cudaError_t launch_index_t(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                  const IndexParams &ip, int grid, cudaStream_t st) {
+    const size_t smem = prefill_index_smem_bytes(D_IDX);
+    cudaFuncSetAttribute(prefill_index_kernel<D_IDX, CAP>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    prefill_index_kernel<D_IDX, CAP><<<grid, 192, smem, st>>>(tm_q, tm_k, ip);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                                 int32_t *ids, int *status, int num_sms, cudaStream_t st) {
+    IndexParams ip;
+    ip.ids = ids;
+    ip.status = status;
+    ip.Bt = sh.Bt;
+    ip.n_q = sh.n_q;
+    ip.T = sh.T;
+    ip.block = sh.block;
+    ip.K = sh.K;
+    ip.n_qt = (sh.n_q + 127) / 128;
+    ip.n_items = ip.n_qt * sh.Bt;
+    const int grid = ip.n_items < num_sms ? ip.n_items : num_sms;
+    if (sh.d_idx == 128) {
+        if (sh.K <= 8) return launch_index_t<128, 7>(tm_q, tm_k, ip, grid, st);
+        if (sh.K <= 16) return launch_index_t<128, 15>(tm_q, tm_k, ip, grid, st);
+        return launch_index_t<128, 31>(tm_q, tm_k, ip, grid, st);
+    }
+    if (sh.K <= 8) return launch_index_t<64, 7>(tm_q, tm_k, ip, grid, st);
+    if (sh.K <= 16) return launch_index_t<64, 15>(tm_q, tm_k, ip, grid, st);
+    return launch_index_t<64, 31>(tm_q, tm_k, ip, grid, st);
+}
+
+size_t prefill_attn_smem_bytes(const Shape &sh) {
+    const int NK = sh.block < 128 ? sh.block : 128;
+    const int NS = sh.block / NK;
+    const int KVST = NS > 1 ? 2 : 1;
+    const size_t kv_tile = static_cast<size_t>(NK) * 128 * (sh.d / 64);
+    const size_t q = static_cast<size_t>(sh.d / 64) * kRegionBytes;
+    const size_t pb = static_cast<size_t>((NK + 63) / 64) * kRegionBytes;
+    return 1024 + KVST * 2 * kv_tile + 2 * q + pb + 64 + 256 * 4 + 32;
+}
+
+cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                                const void *q, const int32_t *row_ptr, const int32_t *entries,
+                                const AttnItem *items, int *counters, void *part_o,
+                                float *part_lse, int *status, int num_sms, cudaStream_t st) {
+    AttnParams ap;
+    ap.q = static_cast<const __nv_bfloat16 *>(q);
+    ap.row_ptr = row_ptr;
+    ap.entries = entries;
+    ap.items = items;
+    ap.counters = counters;
+    ap.part_o = static_cast<__nv_bfloat16 *>(part_o);
+    ap.part_lse = part_lse;
+    ap.status = status;
+    ap.Bt = sh.Bt;
+    ap.n_q = sh.n_q;
+    ap.T = sh.T;
+    ap.Hq = sh.Hq;
+    ap.Hkv = sh.Hkv;
+    ap.G = sh.G;
+    ap.block = sh.block;
+    ap.K = sh.K;
+    ap.N = sh.N;
+    ap.NK = sh.block < 128 ? sh.block : 128;
+    ap.NS = sh.block / ap.NK;
+    ap.TOK = 128 / sh.G;
+    ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(sh.d));
+    const size_t smem = prefill_attn_smem_bytes(sh);
+    if (sh.d == 128) {
+        cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+        prefill_attn_kernel<128><<<num_sms, 128, smem, st>>>(tm_k, tm_v, ap);
+    } else {
+        cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+        prefill_attn_kernel<64><<<num_sms, 128, smem, st>>>(tm_k, tm_v, ap);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace msa

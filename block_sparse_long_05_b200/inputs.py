@@ -138,3 +138,37 @@ def sample_rows(w: Workload, n: int, seed: int = 1) -> torch.Tensor:
         if t_early >= t0:
             picked.add(base + (t_early - t0))
     return torch.tensor(sorted(picked), dtype=torch.int64)
+
+
+def random_selection(w: Workload, device="cpu", seed: int = 2) -> torch.Tensor:
+    """A synthetic selection with the structure of the index branch's output
+    (own block always present, min(K, own+1) distinct blocks <= own, ascending,
+    -1 padded) but drawn at random: used to test the sparse branch apart from
+    the index branch.  Returns ids [Bt, n_q, K] int32 on ``device``."""
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    rows = w.Bt * w.n_q
+    ids = torch.full((rows, w.K), -1, dtype=torch.int32, device=dev)
+    t = (w.T - w.n_q) + torch.arange(rows, device=dev) % w.n_q
+    own = torch.div(t, w.block, rounding_mode="floor")
+    step = max(1, (1 << 24) // max(w.n_blocks, 1))
+    for s in range(0, rows, step):
+        e = min(rows, s + step)
+        o = own[s:e]
+        r = torch.rand((e - s, w.n_blocks), generator=gen, device=dev)
+        cols = torch.arange(w.n_blocks, device=dev)[None, :]
+        r = torch.where(cols < o[:, None], r, torch.full_like(r, -1.0))  # candidates j < own
+        kk = min(w.K - 1, w.n_blocks)
+        if kk > 0:
+            val, idx = torch.topk(r, kk, dim=1)
+            idx = torch.where(val >= 0, idx, torch.full_like(idx, -1))
+        else:
+            idx = torch.empty((e - s, 0), dtype=torch.int64, device=dev)
+        sel = torch.cat([idx, o[:, None]], dim=1)
+        big = torch.iinfo(torch.int64).max
+        sel = torch.where(sel < 0, torch.full_like(sel, big), sel)
+        sel, _ = torch.sort(sel, dim=1)
+        sel = torch.where(sel == big, torch.full_like(sel, -1), sel)
+        ids[s:e, :sel.shape[1]] = sel[:, :w.K].to(torch.int32)
+    return ids.view(w.Bt, w.n_q, w.K)

@@ -1,0 +1,198 @@
+"""Python binding of libmsa (the C ABI in include/msa.h), by ctypes.
+
+Argument marshalling only: every step of the MSA hot path runs in the CUDA
+kernels behind the C ABI.  torch supplies device memory and the current CUDA
+stream.  If libmsa.so is missing, every call raises: there is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa.so")
+
+STATUS = {
+    0: "MSA_OK",
+    1: "MSA_ERR_INVALID_ARG",
+    2: "MSA_ERR_UNSUPPORTED",
+    3: "MSA_ERR_WORKSPACE",
+    4: "MSA_ERR_CUDA",
+    5: "MSA_ERR_TIMEOUT",
+    6: "MSA_ERR_BAD_IDS",
+}
+
+EXPORTED = ("msa_workspace_size", "msa_index_topk", "msa_select_invert", "msa_sparse_attn",
+            "msa_device_status", "msa_status_string", "msa_selftest_umma")
+
+
+class MSAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)} ({code})")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libmsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m block_sparse_long_05_b200.build` (needs nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.msa_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I]
+    lib.msa_workspace_size.restype = Z
+    lib.msa_index_topk.argtypes = [P, P, P, I, I, I, I, I, I, P, Z, P]
+    lib.msa_index_topk.restype = I
+    lib.msa_select_invert.argtypes = [P, P, P, I, I, I, I, I, P, Z, P]
+    lib.msa_select_invert.restype = I
+    lib.msa_sparse_attn.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
+    lib.msa_sparse_attn.restype = I
+    lib.msa_device_status.argtypes = [P, P]
+    lib.msa_device_status.restype = I
+    lib.msa_status_string.argtypes = [I]
+    lib.msa_status_string.restype = ctypes.c_char_p
+    lib.msa_selftest_umma.argtypes = [P, P, P, I, I, I, P, P]
+    lib.msa_selftest_umma.restype = I
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise MSAError(fn, code)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def workspace_size(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K) -> int:
+    return int(load_library().msa_workspace_size(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K))
+
+
+class Workspace:
+    """Device scratch for the calls (status word zeroed at creation)."""
+
+    def __init__(self, nbytes: int, device=None):
+        if nbytes <= 0:
+            raise ValueError("workspace size must be positive (unsupported shape?)")
+        self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device or "cuda")
+        off = (-self.buf.data_ptr()) % 256
+        self.view = self.buf[off:off + nbytes]
+        self.view[:256].zero_()
+        self.nbytes = nbytes
+
+    @property
+    def ptr(self) -> int:
+        return self.view.data_ptr()
+
+    @classmethod
+    def for_shape(cls, Bt, n_q, T, Hq, Hkv, d, d_idx, block, K, device=None) -> "Workspace":
+        return cls(workspace_size(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K), device)
+
+
+def index_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, block: int, K: int, ws: Workspace,
+               ids: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """q_idx [Bt, n_q, d_idx], k_idx [Bt, T, d_idx] bf16 -> ids [Bt, n_q, K] int32."""
+    _dev(q_idx, torch.bfloat16, "q_idx")
+    _dev(k_idx, torch.bfloat16, "k_idx")
+    Bt, n_q, d_idx = q_idx.shape
+    T = k_idx.shape[1]
+    if k_idx.shape != (Bt, T, d_idx):
+        raise ValueError(f"k_idx shape {tuple(k_idx.shape)} does not match q_idx")
+    if ids is None:
+        ids = torch.empty((Bt, n_q, K), dtype=torch.int32, device=q_idx.device)
+    _dev(ids, torch.int32, "ids")
+    lib = load_library()
+    _check("msa_index_topk", lib.msa_index_topk(q_idx.data_ptr(), k_idx.data_ptr(), ids.data_ptr(),
+                                                Bt, n_q, T, d_idx, block, K, ws.ptr, ws.nbytes,
+                                                _stream(stream)))
+    return ids
+
+
+def select_invert(ids: torch.Tensor, T: int, block: int, ws: Workspace, stream=None):
+    """ids [Bt, n_q, K] int32 -> (row_ptr [Bt*N+1], entries [Bt*n_q*K]) int32 (CSR)."""
+    _dev(ids, torch.int32, "ids")
+    Bt, n_q, K = ids.shape
+    N = (T + block - 1) // block
+    row_ptr = torch.empty(Bt * N + 1, dtype=torch.int32, device=ids.device)
+    entries = torch.empty(max(Bt * n_q * K, 1), dtype=torch.int32, device=ids.device)
+    lib = load_library()
+    _check("msa_select_invert", lib.msa_select_invert(ids.data_ptr(), row_ptr.data_ptr(),
+                                                      entries.data_ptr(), Bt, n_q, T, block, K,
+                                                      ws.ptr, ws.nbytes, _stream(stream)))
+    return row_ptr, entries
+
+
+def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ids: torch.Tensor, block: int,
+                ws: Workspace, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                stream=None):
+    """q [Bt, n_q, Hq, d], k/v [Bt, T, Hkv, d] bf16, ids [Bt, n_q, K] int32
+    -> (out [Bt, n_q, Hq, d] fp32, lse [Bt, n_q, Hq] fp32)."""
+    _dev(q, torch.bfloat16, "q")
+    _dev(k, torch.bfloat16, "k")
+    _dev(v, torch.bfloat16, "v")
+    _dev(ids, torch.int32, "ids")
+    Bt, n_q, Hq, d = q.shape
+    T, Hkv = k.shape[1], k.shape[2]
+    if k.shape != (Bt, T, Hkv, d) or v.shape != k.shape:
+        raise ValueError("k/v shapes do not match q")
+    K = ids.shape[-1]
+    if ids.shape != (Bt, n_q, K):
+        raise ValueError("ids shape does not match q")
+    if out is None:
+        out = torch.empty((Bt, n_q, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((Bt, n_q, Hq), dtype=torch.float32, device=q.device)
+    _dev(out, torch.float32, "out")
+    _dev(lse, torch.float32, "lse")
+    lib = load_library()
+    _check("msa_sparse_attn", lib.msa_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                  ids.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                                  Bt, n_q, T, Hq, Hkv, d, block, K, ws.ptr,
+                                                  ws.nbytes, _stream(stream)))
+    return out, lse
+
+
+def device_status(ws: Workspace, stream=None) -> int:
+    """Synchronise the stream, read and clear the workspace's device status."""
+    return int(load_library().msa_device_status(ws.ptr, _stream(stream)))
+
+
+def status_string(code: int) -> str:
+    return load_library().msa_status_string(int(code)).decode()
+
+
+def selftest_umma(A: torch.Tensor, B: torch.Tensor, b_mn_major: bool, stream=None):
+    """C[128, N] = A[128, Kd] @ B with B as [N, Kd] (K-major) or [Kd, N] (MN-major)."""
+    _dev(A, torch.bfloat16, "A")
+    _dev(B, torch.bfloat16, "B")
+    Kd = A.shape[1]
+    N = B.shape[1] if b_mn_major else B.shape[0]
+    C = torch.empty((128, N), dtype=torch.float32, device=A.device)
+    status = torch.zeros(1, dtype=torch.int32, device=A.device)
+    lib = load_library()
+    _check("msa_selftest_umma", lib.msa_selftest_umma(A.data_ptr(), B.data_ptr(), C.data_ptr(), N,
+                                                      Kd, int(b_mn_major), status.data_ptr(),
+                                                      _stream(stream)))
+    return C, status

@@ -1,0 +1,157 @@
+/*
+ * msa.h -- C ABI of libmsa: the hot path of MiniMax Sparse Attention (MSA)
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The method (web pages, cited by title and section):
+ *   [P2] "MiniMax M3模型算力成本大幅降低原因深度解析", sections "索引分支（Index
+ *        Branch）" and "稀疏分支（Sparse Branch）": a lightweight single-head
+ *        index key with block max-pooling screens the whole context and keeps
+ *        the top-K KV blocks; standard GQA then runs over the kept blocks only,
+ *        on raw KV.
+ *   [P4] "MiniMax M3 深度实战 ...", section 2.2 "KV Outer Gather Q" (each KV
+ *        block gathers the queries that selected it and is read once), section
+ *        2.3 "MSA 算法实现" (the own/local block is always kept; softmax of
+ *        Q K^T / sqrt(d_head) over the gathered keys), section 3.3 (decode:
+ *        one new query, at the newest position).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates, frees or retains memory; it keeps no global mutable
+ *    state, so calls on different workspaces may run concurrently.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *    asynchronous on that stream and returns after enqueueing its kernels.
+ *  - Layouts are row-major and contiguous, bf16 means IEEE bfloat16 bits:
+ *        q_idx [Bt][n_q][d_idx]  bf16     k_idx [Bt][T][d_idx]   bf16
+ *        q     [Bt][n_q][Hq][d]  bf16     k, v  [Bt][T][Hkv][d]  bf16
+ *        ids   [Bt][n_q][K]      int32    out   [Bt][n_q][Hq][d] fp32
+ *        lse   [Bt][n_q][Hq]     fp32
+ *    Query i (0 <= i < n_q) of sequence b sits at position t = T - n_q + i of
+ *    its length-T context (prefill: n_q = T; decode: n_q = 1).  Block j holds
+ *    keys [j*block, min((j+1)*block, T)); N = ceil(T / block); own(t) = t / block.
+ *  - Selection: ids[b][i] lists min(K, own(t)+1) distinct blocks in ascending
+ *    order, padded with -1: the own block, plus the top min(K, own+1) - 1 of
+ *    the blocks j < own(t) ranked by s(t,j) = max_{i in block j} q_idx[t].k_idx[i]
+ *    (descending; ties go to the lower block index).  Scores are accumulated in
+ *    fp32, which is exact for the integer-valued index keys of the pages'
+ *    workloads (|s| < 2^24).
+ *  - Attention: for each query head h (kv head h / (Hq/Hkv)), softmax of
+ *    q.k_i / sqrt(d) over the keys i <= t of the blocks in ids, output the
+ *    weighted sum of v_i (fp32) and lse = ln sum_i exp(q.k_i / sqrt(d)).
+ *  - Supported shapes: d, d_idx in {64, 128}; block in {32, 64} or a
+ *    multiple of 128; 1 <= K <= 32; 128 % (Hq/Hkv) == 0; N <= 8192 for
+ *    prefill (n_q > 1); Bt*T < 2^31 and Bt*n_q*K < 2^31.  Anything else
+ *    returns MSA_ERR_UNSUPPORTED before any work is enqueued.  Tensor base
+ *    pointers must be 16-byte aligned (MSA_ERR_INVALID_ARG otherwise).
+ *  - Errors found on the host return immediately (nothing enqueued).  Errors a
+ *    kernel finds (an id outside [-1, N), a bounded wait that expired) are
+ *    OR-ed into a sticky status word at the start of the workspace; kernels
+ *    skip the offending work and never trap.  Read it with msa_device_status().
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum msa_status {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, n_q > T, Hq % Hkv != 0, K < 1 */
+    MSA_ERR_UNSUPPORTED = 2, /* valid but outside the supported shapes listed above */
+    MSA_ERR_WORKSPACE = 3,   /* workspace pointer null/misaligned or smaller than required */
+    MSA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    MSA_ERR_TIMEOUT = 5,     /* device: a bounded wait inside a kernel expired */
+    MSA_ERR_BAD_IDS = 6      /* device: an id outside [-1, N) was seen and skipped */
+} msa_status;
+
+/*
+ * Bytes of device workspace that msa_index_topk, msa_select_invert and
+ * msa_sparse_attn need for these sizes (the maximum over the three; a decode
+ * shape, n_q == 1, needs far less than a prefill).  The workspace must be
+ * 256-byte aligned.  Its first 256 bytes hold the sticky device status word:
+ * zero them once before first use (e.g. cudaMemsetAsync(ws, 0, 256)).  The
+ * rest is scratch that every call overwrites; two calls that overlap in time
+ * must not share a workspace.  Returns 0 for arguments the calls would reject.
+ */
+MSA_API size_t msa_workspace_size(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_idx, int block,
+                          int K);
+
+/*
+ * Index branch [P2 "索引分支"]: block max-pooled single-head index scores and
+ * top-K block selection with the own block forced.  Writes ids (layout above).
+ * Prefill (n_q > 1) runs one fused tcgen05 kernel that never materialises the
+ * n_q x T score matrix; decode (n_q == 1) streams k_idx once and selects.
+ */
+MSA_API msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t *ids, int Bt, int n_q,
+                          int T, int d_idx, int block, int K, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/*
+ * Selection inversion [P4 section 2.2]: the per-query block lists in ids
+ * turned into per-block lists of hit queries, in CSR form over the Bt*N
+ * (sequence, block) pairs:
+ *   row_ptr [Bt*N + 1] int32: list of pair p = b*N + j is
+ *           entries[row_ptr[p] .. row_ptr[p+1]);
+ *   entries [Bt*n_q*K] int32 (capacity; row_ptr[Bt*N] are used): each entry
+ *           is (b*n_q + i)*K + slot with ids[b][i][slot] == j, listed in
+ *           ascending query order.
+ * msa_sparse_attn performs the same inversion internally (into its
+ * workspace); this entry point exposes it on its own.
+ */
+MSA_API msa_status msa_select_invert(const int32_t *ids, int32_t *row_ptr, int32_t *entries, int Bt,
+                             int n_q, int T, int block, int K, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/*
+ * Sparse branch [P2 "稀疏分支"; P4 sections 2.2, 2.3]: exact GQA softmax
+ * attention over the keys of the selected blocks (causal inside the own block),
+ * scale 1/sqrt(d), raw bf16 KV.  Writes out and lse (layouts above).
+ * ids must hold, per row, distinct block ids in [0, N) or -1; an id greater
+ * than own(t) contributes no key.  Prefill (n_q > 1): inversion, a
+ * KV-block-outer tcgen05 kernel that loads each selected KV block into shared
+ * memory and gathers its hit queries, then a log-sum-exp combine of the per
+ * slot partials.  Decode (n_q == 1): a split-K kernel over the selected blocks,
+ * then the same combine.
+ */
+MSA_API msa_status msa_sparse_attn(const void *q, const void *k, const void *v, const int32_t *ids,
+                           float *out, float *lse, int Bt, int n_q, int T, int Hq, int Hkv, int d,
+                           int block, int K, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the sticky device status word
+ * of `workspace`: MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_BAD_IDS (the first found,
+ * in that order of precedence: timeout first), or MSA_ERR_CUDA if the
+ * synchronisation or the copy failed.
+ */
+MSA_API msa_status msa_device_status(void *workspace, void *stream);
+
+/* Static, NUL-terminated name of a status code ("unknown status" otherwise). */
+MSA_API const char *msa_status_string(int status);
+
+/*
+ * Tensor-core self-test, not part of the method: C[128][N] = A . B with
+ * A [128][Kd] bf16 (K-major) and B either as [N][Kd] (b_mn_major = 0, K-major)
+ * or as [Kd][N] (b_mn_major = 1), C fp32, through the same TMA, shared-memory
+ * descriptor, tcgen05.mma and TMEM read-back code the attention kernels use.
+ * N in {64, 128, 256}, Kd a multiple of 64 up to 256.  Device pointers;
+ * `status` is a device int the kernel sets non-zero on a wait timeout.
+ */
+MSA_API msa_status msa_selftest_umma(const void *A, const void *B, float *C, int N, int Kd,
+                             int b_mn_major, int *status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H */

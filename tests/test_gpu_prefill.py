@@ -1,0 +1,145 @@
+"""Prefill path (n_q > 1) of the CUDA library against the CPU oracle:
+tcgen05 index kernel (bit-exact ids), selection inversion (bit-exact CSR),
+KV-block-outer tcgen05 attention + log-sum-exp combine (within tolerance).
+Small shapes are checked on every row; the full-size workloads on sampled
+rows (uniform, seed 1, plus each sequence's first, last and a dense-early
+row)."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import assert_close, host, lib_ready, rows_of, run_attn, run_index
+
+pytestmark = pytest.mark.gpu
+
+from block_sparse_long_05_b200.inputs import (PREFILL_256K, PREFILL_64K, TINY_PREFILL, Workload,
+                                              make_inputs, random_selection, sample_rows)
+
+N_SAMPLE = int(os.environ.get("MSA_TEST_SAMPLE_ROWS", "4096"))
+
+
+def _ws(w):
+    from block_sparse_long_05_b200 import msa
+    return msa.Workspace.for_shape(w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K)
+
+
+def _check_ids(w, x, ids, rows):
+    from oracle import oracle
+    exp = oracle.index_topk(host(x["q_idx"]), host(x["k_idx"]), w.Bt, w.n_q, w.T, w.d_idx,
+                            w.block, w.K, rows=rows.numpy())
+    got = host(rows_of(ids, rows, w.K)).numpy()
+    bad = np.nonzero(~np.all(got == exp, axis=1))[0]
+    assert bad.size == 0, f"{bad.size} rows differ, first row {int(rows[bad[0]])}: " \
+                          f"{got[bad[0]]} vs {exp[bad[0]]}"
+    return exp
+
+
+def _check_attn(w, x, ids_rows, out, lse, rows):
+    from oracle import oracle
+    hq, hk, hv = host(x["q"]), host(x["k"]), host(x["v"])
+    o_ref, l_ref = oracle.sparse_attn(hq, hk, hv, ids_rows, w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d,
+                                      w.block, w.K, rows=rows.numpy())
+    assert_close(host(rows_of(out, rows, 0)).numpy(), o_ref, "out")
+    assert_close(host(rows_of(lse, rows, 0)).numpy(), l_ref, "lse")
+
+
+def _end_to_end(w, rows=None, index_values="int3"):
+    lib_ready()
+    x = make_inputs(w, device="cuda", index_values=index_values)
+    ws = _ws(w)
+    ids = run_index(w, x, ws)
+    if rows is None:
+        rows = torch.arange(w.Bt * w.n_q, dtype=torch.int64)
+    ids_ref = _check_ids(w, x, ids, rows)
+    out, lse = run_attn(w, x, ids, ws)
+    _check_attn(w, x, ids_ref, out, lse, rows)
+
+
+SMALL = [
+    Workload("pf_tiny_b64", 1, 512, 512, 8, 2, 64, 64, 4, 64),
+    Workload("pf_ragged", 2, 1000, 1000, 8, 2, 64, 64, 4, 64),        # T % block != 0, Bt = 2
+    Workload("pf_b128_d128", 1, 2048, 2048, 16, 2, 128, 128, 8, 128),
+    Workload("pf_b256", 1, 2048, 2048, 8, 1, 128, 256, 4, 128),       # streamed KV sub-tiles, G=8
+    Workload("pf_b512", 1, 3000, 3000, 8, 4, 128, 512, 3, 64),        # ragged, 4 sub-tiles
+    Workload("pf_b32_k32", 1, 1500, 1500, 4, 4, 64, 32, 32, 64),      # G = 1, K = 32
+    Workload("pf_dense", 1, 700, 700, 8, 2, 64, 64, 16, 128),         # K >= N: dense causal
+    Workload("pf_k1", 2, 600, 600, 8, 2, 128, 64, 1, 64),             # own block only
+    Workload("pf_chunk", 2, 300, 2000, 8, 2, 64, 128, 6, 64),         # last n_q queries only
+    Workload("pf_short", 1, 40, 40, 8, 2, 64, 64, 4, 64),             # single block, T < block
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_prefill_small_all_rows(w):
+    _end_to_end(w)
+
+
+def test_prefill_index_ties():
+    _end_to_end(Workload("pf_ties", 1, 1024, 1024, 8, 2, 64, 64, 5, 64), index_values="zeros")
+
+
+def test_prefill_tiny_workload_all_rows():
+    _end_to_end(TINY_PREFILL)
+
+
+@pytest.mark.parametrize("w", [SMALL[1], SMALL[3], SMALL[4], SMALL[8]], ids=lambda w: w.name)
+def test_inversion_exact(w):
+    from block_sparse_long_05_b200 import msa
+    from oracle import oracle
+    lib_ready()
+    ids = random_selection(w, device="cuda")
+    ws = _ws(w)
+    row_ptr, entries = msa.select_invert(ids, w.T, w.block, ws)
+    assert msa.device_status(ws) == 0
+    rp_ref, ent_ref = oracle.select_invert(host(ids), w.Bt, w.n_q, w.T, w.block, w.K)
+    rp = host(row_ptr).numpy()
+    assert np.array_equal(rp, rp_ref)
+    assert np.array_equal(host(entries).numpy()[: rp[-1]], ent_ref)
+
+
+def test_inversion_full_size():
+    from block_sparse_long_05_b200 import msa
+    from oracle import oracle
+    lib_ready()
+    w = PREFILL_256K
+    ids = random_selection(w, device="cuda")
+    ws = msa.Workspace(1 << 28)
+    row_ptr, entries = msa.select_invert(ids, w.T, w.block, ws)
+    assert msa.device_status(ws) == 0
+    rp_ref, ent_ref = oracle.select_invert(host(ids), w.Bt, w.n_q, w.T, w.block, w.K)
+    rp = host(row_ptr).numpy()
+    assert np.array_equal(rp, rp_ref)
+    assert np.array_equal(host(entries).numpy()[: rp[-1]], ent_ref)
+
+
+@pytest.mark.parametrize("w", [SMALL[2], SMALL[4], SMALL[5]], ids=lambda w: w.name)
+def test_attention_random_selection(w):
+    # the sparse branch alone, on a seeded random selection of the same structure
+    lib_ready()
+    x = make_inputs(w, device="cuda")
+    ids = random_selection(w, device="cuda")
+    out, lse = run_attn(w, x, ids, _ws(w))
+    rows = torch.arange(w.Bt * w.n_q, dtype=torch.int64)
+    _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)
+
+
+@pytest.mark.parametrize("w", [PREFILL_64K, PREFILL_256K], ids=lambda w: w.name)
+def test_prefill_full_size_sampled(w):
+    _end_to_end(w, rows=sample_rows(w, N_SAMPLE))
+    torch.cuda.empty_cache()
+
+
+def test_prefill_bad_ids_reported():
+    from block_sparse_long_05_b200 import msa
+    lib_ready()
+    w = Workload("pf_bad", 1, 256, 256, 8, 2, 64, 64, 2, 64)
+    x = make_inputs(w, device="cuda")
+    ids = random_selection(w, device="cuda")
+    ids[0, 5, 1] = 77      # beyond N = 4
+    ids[0, 9, 1] = -3
+    ws = _ws(w)
+    out, lse = msa.sparse_attn(x["q"], x["k"], x["v"], ids, w.block, ws)
+    assert msa.device_status(ws) == 6  # MSA_ERR_BAD_IDS
+    assert torch.isfinite(out[0, 100]).all()
