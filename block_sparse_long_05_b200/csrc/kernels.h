@@ -12,8 +12,10 @@
 namespace msa {
 
 // SIMT kernels (kernels_simt.cu)
-cudaError_t launch_decode_index(const Shape &sh, const void *q_idx, const void *k_idx,
-                                int32_t *ids, float *block_scores, int num_sms, cudaStream_t st);
+cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k_idx,
+                               float *block_scores, int num_sms, cudaStream_t st);
+cudaError_t launch_decode_select(const Shape &sh, const float *block_scores, int32_t *ids,
+                                 cudaStream_t st);
 size_t decode_attn_smem_bytes(const Shape &sh);
 cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, const void *v,
                                const int32_t *ids, float *part_o, float *part_lse, int S,

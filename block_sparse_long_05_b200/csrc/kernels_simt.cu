@@ -539,9 +539,8 @@ __global__ void __launch_bounds__(256) attn_items_kernel(const int *__restrict__
 }  // namespace
 
 // ------------------------------------------------------------------ launchers
-cudaError_t launch_decode_index(const Shape &sh, const void *q_idx, const void *k_idx,
-                                int32_t *ids, float *block_scores, int num_sms,
-                                cudaStream_t st) {
+cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k_idx,
+                               float *block_scores, int num_sms, cudaStream_t st) {
     const int own = (sh.T - 1) / sh.block;
     if (own > 0) {
         const long long work = static_cast<long long>(sh.Bt) * own;
@@ -557,6 +556,12 @@ cudaError_t launch_decode_index(const Shape &sh, const void *q_idx, const void *
             decode_index_scan_kernel<64><<<static_cast<int>(blocks), 256, 0, st>>>(
                 qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_select(const Shape &sh, const float *block_scores, int32_t *ids,
+                                 cudaStream_t st) {
+    const int own = (sh.T - 1) / sh.block;
     if (sh.K <= 8)
         decode_select_kernel<7><<<sh.Bt, 32, 0, st>>>(block_scores, ids, sh.N, own, sh.K);
     else if (sh.K <= 16)

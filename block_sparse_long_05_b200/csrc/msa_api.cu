@@ -143,6 +143,13 @@ bool make_tmap(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dim
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Record the start/stop event of stage i (if the caller supplied one).
+void mark(const msa_stage_events *ev, int i, bool start, cudaStream_t st) {
+    if (!ev) return;
+    void *e = start ? ev->start[i] : ev->stop[i];
+    if (e) cudaEventRecord(static_cast<cudaEvent_t>(e), st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -157,6 +164,13 @@ size_t msa_workspace_size(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_
 msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t *ids, int Bt, int n_q,
                           int T, int d_idx, int block, int K, void *workspace,
                           size_t workspace_bytes, void *stream) {
+    return msa_index_topk_ev(q_idx, k_idx, ids, Bt, n_q, T, d_idx, block, K, workspace,
+                             workspace_bytes, stream, nullptr);
+}
+
+msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids, int Bt, int n_q,
+                             int T, int d_idx, int block, int K, void *workspace,
+                             size_t workspace_bytes, void *stream, const msa_stage_events *ev) {
     if (!q_idx || !k_idx || !ids) return MSA_ERR_INVALID_ARG;
     Shape sh;
     msa_status s = validate(Bt, n_q, T, 1, 1, 64, d_idx, block, K, true, false, &sh);
@@ -168,9 +182,16 @@ msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t *ids, in
     const int sms = num_sms_current();
     if (sms <= 0) return MSA_ERR_CUDA;
     int *status = at<int>(workspace, L.status);
-    if (n_q == 1)
-        return cuda_status(launch_decode_index(sh, q_idx, k_idx, ids, at<float>(workspace, L.block_scores),
-                                               sms, st));
+    if (n_q == 1) {
+        float *scores = at<float>(workspace, L.block_scores);
+        mark(ev, 0, true, st);
+        if (launch_decode_scan(sh, q_idx, k_idx, scores, sms, st) != cudaSuccess) return MSA_ERR_CUDA;
+        mark(ev, 0, false, st);
+        mark(ev, 1, true, st);
+        if (launch_decode_select(sh, scores, ids, st) != cudaSuccess) return MSA_ERR_CUDA;
+        mark(ev, 1, false, st);
+        return MSA_OK;
+    }
     CUtensorMap tq, tk;
     const cuuint64_t dq[2] = {static_cast<cuuint64_t>(d_idx), static_cast<cuuint64_t>(Bt) * n_q};
     const cuuint64_t dk[2] = {static_cast<cuuint64_t>(d_idx), static_cast<cuuint64_t>(Bt) * T};
@@ -178,7 +199,10 @@ msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t *ids, in
     const cuuint32_t box[2] = {64, 128};
     if (!make_tmap(&tq, q_idx, 2, dq, str, box) || !make_tmap(&tk, k_idx, 2, dk, str, box))
         return MSA_ERR_CUDA;
-    return cuda_status(launch_prefill_index(sh, tq, tk, ids, status, sms, st));
+    mark(ev, 0, true, st);
+    const cudaError_t e = launch_prefill_index(sh, tq, tk, ids, status, sms, st);
+    mark(ev, 0, false, st);
+    return cuda_status(e);
 }
 
 msa_status msa_select_invert(const int32_t *ids, int32_t *row_ptr, int32_t *entries, int Bt,
@@ -202,6 +226,14 @@ msa_status msa_sparse_attn(const void *q, const void *k, const void *v, const in
                            float *out, float *lse, int Bt, int n_q, int T, int Hq, int Hkv, int d,
                            int block, int K, void *workspace, size_t workspace_bytes,
                            void *stream) {
+    return msa_sparse_attn_ev(q, k, v, ids, out, lse, Bt, n_q, T, Hq, Hkv, d, block, K, workspace,
+                              workspace_bytes, stream, nullptr);
+}
+
+msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const int32_t *ids,
+                              float *out, float *lse, int Bt, int n_q, int T, int Hq, int Hkv,
+                              int d, int block, int K, void *workspace, size_t workspace_bytes,
+                              void *stream, const msa_stage_events *ev) {
     if (!q || !k || !v || !ids || !out || !lse) return MSA_ERR_INVALID_ARG;
     Shape sh;
     msa_status s = validate(Bt, n_q, T, Hq, Hkv, d, 64, block, K, false, true, &sh);
@@ -215,9 +247,14 @@ msa_status msa_sparse_attn(const void *q, const void *k, const void *v, const in
         const int S = L.decode_splits;
         float *po = at<float>(workspace, L.part_o);
         float *pl = at<float>(workspace, L.part_lse);
+        mark(ev, 1, true, st);
         cudaError_t e = launch_decode_attn(sh, q, k, v, ids, po, pl, S, status, st);
         if (e != cudaSuccess) return MSA_ERR_CUDA;
-        return cuda_status(launch_combine(sh, po, false, pl, ids, out, lse, S, st));
+        mark(ev, 1, false, st);
+        mark(ev, 2, true, st);
+        e = launch_combine(sh, po, false, pl, ids, out, lse, S, st);
+        mark(ev, 2, false, st);
+        return cuda_status(e);
     }
     const int sms = num_sms_current();
     if (sms <= 0) return MSA_ERR_CUDA;
@@ -225,11 +262,13 @@ msa_status msa_sparse_attn(const void *q, const void *k, const void *v, const in
     int32_t *ent = at<int32_t>(workspace, L.entries);
     AttnItem *items = at<AttnItem>(workspace, L.items);
     int *counters = at<int>(workspace, L.counters);
+    mark(ev, 0, true, st);
     cudaError_t e = launch_invert(sh, ids, at<int>(workspace, L.chunk_counts),
                                   at<int>(workspace, L.pair_totals), rp, ent,
                                   at<int>(workspace, L.item_ptr), items, counters,
                                   L.rows_per_item, L.n_chunks, status, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
+    mark(ev, 0, false, st);
     const int NK = block < 128 ? block : 128;
     CUtensorMap tk, tv;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Hkv),
@@ -240,9 +279,14 @@ msa_status msa_sparse_attn(const void *q, const void *k, const void *v, const in
         return MSA_ERR_CUDA;
     void *po = at<void>(workspace, L.part_o);
     float *pl = at<float>(workspace, L.part_lse);
+    mark(ev, 1, true, st);
     e = launch_prefill_attn(sh, tk, tv, q, rp, ent, items, counters, po, pl, status, sms, st);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
-    return cuda_status(launch_combine(sh, po, true, pl, ids, out, lse, 1, st));
+    mark(ev, 1, false, st);
+    mark(ev, 2, true, st);
+    e = launch_combine(sh, po, true, pl, ids, out, lse, 1, st);
+    mark(ev, 2, false, st);
+    return cuda_status(e);
 }
 
 msa_status msa_device_status(void *workspace, void *stream) {

@@ -63,7 +63,15 @@ DECODE_128K = Workload("decode_32x131072", 32, 1, 131072, 64, 8, 128, 128, 16, 1
 PREFILL_256K = Workload("long_prefill_T262144", 1, 262144, 262144, 64, 8, 128, 512, 8, 128)
 DECODE_1M = Workload("decode_4x1048576", 4, 1, 1048576, 64, 8, 128, 512, 8, 128)
 
-WORKLOADS = {w.name: w for w in (TINY_PREFILL, PREFILL_64K, DECODE_128K, PREFILL_256K, DECODE_1M)}
+# Smaller cases with the same head layout, for profiler captures (inputs still
+# larger than the 126 MB L2, a few GB on the device in total).
+PROFILE_PREFILL = Workload("profile_prefill_T16384", 1, 16384, 16384, 32, 8, 128, 128, 16, 128)
+PROFILE_LONG_PREFILL = Workload("profile_long_prefill_T32768", 1, 32768, 32768, 64, 8, 128, 512,
+                                8, 128)
+PROFILE_DECODE = Workload("profile_decode_4x131072", 4, 1, 131072, 64, 8, 128, 512, 8, 128)
+
+WORKLOADS = {w.name: w for w in (TINY_PREFILL, PREFILL_64K, DECODE_128K, PREFILL_256K, DECODE_1M,
+                                 PROFILE_PREFILL, PROFILE_LONG_PREFILL, PROFILE_DECODE)}
 
 
 def _fill_normal(out: torch.Tensor, gen: torch.Generator) -> None:

@@ -25,7 +25,33 @@ STATUS = {
 }
 
 EXPORTED = ("msa_workspace_size", "msa_index_topk", "msa_select_invert", "msa_sparse_attn",
-            "msa_device_status", "msa_status_string", "msa_selftest_umma")
+            "msa_index_topk_ev", "msa_sparse_attn_ev", "msa_device_status", "msa_status_string",
+            "msa_selftest_umma")
+
+MAX_STAGES = 4
+
+
+class StageEvents(ctypes.Structure):
+    """msa_stage_events: cudaEvent_t handles recorded around each stage."""
+    _fields_ = [("start", ctypes.c_void_p * MAX_STAGES), ("stop", ctypes.c_void_p * MAX_STAGES)]
+
+
+def _event_handle(ev) -> int:
+    """Raw cudaEvent_t of a torch.cuda.Event (created on first record)."""
+    if ev.cuda_event == 0:
+        ev.record()
+    return ev.cuda_event
+
+
+def _stage_events(events):
+    """events: {stage: (start torch.cuda.Event, stop torch.cuda.Event)} or None."""
+    if not events:
+        return None
+    se = StageEvents()
+    for i, (a, b) in events.items():
+        se.start[i] = _event_handle(a) if a is not None else None
+        se.stop[i] = _event_handle(b) if b is not None else None
+    return ctypes.byref(se)
 
 
 class MSAError(RuntimeError):
@@ -59,6 +85,10 @@ def load_library(path: str = LIB_PATH):
     lib.msa_device_status.restype = I
     lib.msa_status_string.argtypes = [I]
     lib.msa_status_string.restype = ctypes.c_char_p
+    lib.msa_index_topk_ev.argtypes = [P, P, P, I, I, I, I, I, I, P, Z, P, P]
+    lib.msa_index_topk_ev.restype = I
+    lib.msa_sparse_attn_ev.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P, P]
+    lib.msa_sparse_attn_ev.restype = I
     lib.msa_selftest_umma.argtypes = [P, P, P, I, I, I, P, P]
     lib.msa_selftest_umma.restype = I
     _lib = lib
@@ -112,8 +142,9 @@ class Workspace:
 
 
 def index_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, block: int, K: int, ws: Workspace,
-               ids: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """q_idx [Bt, n_q, d_idx], k_idx [Bt, T, d_idx] bf16 -> ids [Bt, n_q, K] int32."""
+               ids: torch.Tensor | None = None, stream=None, events=None) -> torch.Tensor:
+    """q_idx [Bt, n_q, d_idx], k_idx [Bt, T, d_idx] bf16 -> ids [Bt, n_q, K] int32.
+    events: optional {stage: (start, stop)} torch.cuda.Event pairs (msa_index_topk_ev)."""
     _dev(q_idx, torch.bfloat16, "q_idx")
     _dev(k_idx, torch.bfloat16, "k_idx")
     Bt, n_q, d_idx = q_idx.shape
@@ -124,9 +155,10 @@ def index_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, block: int, K: int, ws:
         ids = torch.empty((Bt, n_q, K), dtype=torch.int32, device=q_idx.device)
     _dev(ids, torch.int32, "ids")
     lib = load_library()
-    _check("msa_index_topk", lib.msa_index_topk(q_idx.data_ptr(), k_idx.data_ptr(), ids.data_ptr(),
-                                                Bt, n_q, T, d_idx, block, K, ws.ptr, ws.nbytes,
-                                                _stream(stream)))
+    _check("msa_index_topk", lib.msa_index_topk_ev(q_idx.data_ptr(), k_idx.data_ptr(),
+                                                   ids.data_ptr(), Bt, n_q, T, d_idx, block, K,
+                                                   ws.ptr, ws.nbytes, _stream(stream),
+                                                   _stage_events(events)))
     return ids
 
 
@@ -146,9 +178,10 @@ def select_invert(ids: torch.Tensor, T: int, block: int, ws: Workspace, stream=N
 
 def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ids: torch.Tensor, block: int,
                 ws: Workspace, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
-                stream=None):
+                stream=None, events=None):
     """q [Bt, n_q, Hq, d], k/v [Bt, T, Hkv, d] bf16, ids [Bt, n_q, K] int32
-    -> (out [Bt, n_q, Hq, d] fp32, lse [Bt, n_q, Hq] fp32)."""
+    -> (out [Bt, n_q, Hq, d] fp32, lse [Bt, n_q, Hq] fp32).
+    events: optional {stage: (start, stop)} torch.cuda.Event pairs (msa_sparse_attn_ev)."""
     _dev(q, torch.bfloat16, "q")
     _dev(k, torch.bfloat16, "k")
     _dev(v, torch.bfloat16, "v")
@@ -167,10 +200,11 @@ def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ids: torch.Te
     _dev(out, torch.float32, "out")
     _dev(lse, torch.float32, "lse")
     lib = load_library()
-    _check("msa_sparse_attn", lib.msa_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                                  ids.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                                  Bt, n_q, T, Hq, Hkv, d, block, K, ws.ptr,
-                                                  ws.nbytes, _stream(stream)))
+    _check("msa_sparse_attn", lib.msa_sparse_attn_ev(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                     ids.data_ptr(), out.data_ptr(),
+                                                     lse.data_ptr(), Bt, n_q, T, Hq, Hkv, d,
+                                                     block, K, ws.ptr, ws.nbytes,
+                                                     _stream(stream), _stage_events(events)))
     return out, lse
 
 

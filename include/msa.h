@@ -83,8 +83,8 @@ typedef enum msa_status {
  * rest is scratch that every call overwrites; two calls that overlap in time
  * must not share a workspace.  Returns 0 for arguments the calls would reject.
  */
-MSA_API size_t msa_workspace_size(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_idx, int block,
-                          int K);
+MSA_API size_t msa_workspace_size(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_idx,
+                                  int block, int K);
 
 /*
  * Index branch [P2 "索引分支"]: block max-pooled single-head index scores and
@@ -92,9 +92,9 @@ MSA_API size_t msa_workspace_size(int Bt, int n_q, int T, int Hq, int Hkv, int d
  * Prefill (n_q > 1) runs one fused tcgen05 kernel that never materialises the
  * n_q x T score matrix; decode (n_q == 1) streams k_idx once and selects.
  */
-MSA_API msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t *ids, int Bt, int n_q,
-                          int T, int d_idx, int block, int K, void *workspace,
-                          size_t workspace_bytes, void *stream);
+MSA_API msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t *ids, int Bt,
+                                  int n_q, int T, int d_idx, int block, int K, void *workspace,
+                                  size_t workspace_bytes, void *stream);
 
 /*
  * Selection inversion [P4 section 2.2]: the per-query block lists in ids
@@ -108,9 +108,9 @@ MSA_API msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t 
  * msa_sparse_attn performs the same inversion internally (into its
  * workspace); this entry point exposes it on its own.
  */
-MSA_API msa_status msa_select_invert(const int32_t *ids, int32_t *row_ptr, int32_t *entries, int Bt,
-                             int n_q, int T, int block, int K, void *workspace,
-                             size_t workspace_bytes, void *stream);
+MSA_API msa_status msa_select_invert(const int32_t *ids, int32_t *row_ptr, int32_t *entries,
+                                     int Bt, int n_q, int T, int block, int K, void *workspace,
+                                     size_t workspace_bytes, void *stream);
 
 /*
  * Sparse branch [P2 "稀疏分支"; P4 sections 2.2, 2.3]: exact GQA softmax
@@ -123,10 +123,39 @@ MSA_API msa_status msa_select_invert(const int32_t *ids, int32_t *row_ptr, int32
  * slot partials.  Decode (n_q == 1): a split-K kernel over the selected blocks,
  * then the same combine.
  */
-MSA_API msa_status msa_sparse_attn(const void *q, const void *k, const void *v, const int32_t *ids,
-                           float *out, float *lse, int Bt, int n_q, int T, int Hq, int Hkv, int d,
-                           int block, int K, void *workspace, size_t workspace_bytes,
-                           void *stream);
+MSA_API msa_status msa_sparse_attn(const void *q, const void *k, const void *v,
+                                   const int32_t *ids, float *out, float *lse, int Bt, int n_q,
+                                   int T, int Hq, int Hkv, int d, int block, int K,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Instrumented variants (profiling): the same work as msa_index_topk and
+ * msa_sparse_attn, with optional CUDA events recorded on `stream`
+ * immediately before (start[i]) and after (stop[i]) the kernels of stage i.
+ * Each non-NULL entry must be a cudaEvent_t created on the current device;
+ * `events` itself may be NULL.  Stages:
+ *   msa_index_topk_ev:  0 = index kernel (prefill) or k_idx scan (decode);
+ *                       1 = top-K select (decode only).
+ *   msa_sparse_attn_ev: 0 = selection inversion (prefill only);
+ *                       1 = attention kernel (KV-block-outer or split-K);
+ *                       2 = log-sum-exp combine.
+ */
+#define MSA_MAX_STAGES 4
+typedef struct msa_stage_events {
+    void *start[MSA_MAX_STAGES];
+    void *stop[MSA_MAX_STAGES];
+} msa_stage_events;
+
+MSA_API msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids, int Bt,
+                                     int n_q, int T, int d_idx, int block, int K,
+                                     void *workspace, size_t workspace_bytes, void *stream,
+                                     const msa_stage_events *events);
+
+MSA_API msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v,
+                                      const int32_t *ids, float *out, float *lse, int Bt,
+                                      int n_q, int T, int Hq, int Hkv, int d, int block, int K,
+                                      void *workspace, size_t workspace_bytes, void *stream,
+                                      const msa_stage_events *events);
 
 /*
  * Synchronises `stream`, then reads and clears the sticky device status word
@@ -148,7 +177,7 @@ MSA_API const char *msa_status_string(int status);
  * `status` is a device int the kernel sets non-zero on a wait timeout.
  */
 MSA_API msa_status msa_selftest_umma(const void *A, const void *B, float *C, int N, int Kd,
-                             int b_mn_major, int *status, void *stream);
+                                     int b_mn_major, int *status, void *stream);
 
 #ifdef __cplusplus
 }
