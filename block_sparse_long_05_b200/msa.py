@@ -26,7 +26,7 @@ STATUS = {
 
 EXPORTED = ("msa_workspace_size", "msa_index_topk", "msa_select_invert", "msa_sparse_attn",
             "msa_index_topk_ev", "msa_sparse_attn_ev", "msa_device_status", "msa_status_string",
-            "msa_selftest_umma")
+            "msa_selftest_umma", "msa_sparse_attn_decode_noalloc")
 
 MAX_STAGES = 4
 
@@ -89,6 +89,8 @@ def load_library(path: str = LIB_PATH):
     lib.msa_index_topk_ev.restype = I
     lib.msa_sparse_attn_ev.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P, P]
     lib.msa_sparse_attn_ev.restype = I
+    lib.msa_sparse_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
+    lib.msa_sparse_attn_decode_noalloc.restype = I
     lib.msa_selftest_umma.argtypes = [P, P, P, I, I, I, P, P]
     lib.msa_selftest_umma.restype = I
     _lib = lib
@@ -205,6 +207,41 @@ def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ids: torch.Te
                                                      lse.data_ptr(), Bt, n_q, T, Hq, Hkv, d,
                                                      block, K, ws.ptr, ws.nbytes,
                                                      _stream(stream), _stage_events(events)))
+    return out, lse
+
+
+def sparse_attn_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                               ids: torch.Tensor, block: int, out: torch.Tensor | None = None,
+                               lse: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                               stream=None):
+    """Decode attention (n_q = 1) whose scratch is the library's static device
+    array (msa_sparse_attn_decode_noalloc): no workspace is passed and the
+    library allocates nothing.  q [Bt, 1, Hq, d], k/v [Bt, T, Hkv, d] bf16,
+    ids [Bt, 1, K] int32 -> (out [Bt, 1, Hq, d], lse [Bt, 1, Hq]) fp32.
+    status: optional int32 CUDA tensor of one element that receives error bits."""
+    _dev(q, torch.bfloat16, "q")
+    _dev(k, torch.bfloat16, "k")
+    _dev(v, torch.bfloat16, "v")
+    _dev(ids, torch.int32, "ids")
+    Bt, n_q, Hq, d = q.shape
+    if n_q != 1:
+        raise ValueError("the no-allocation entry point serves decode steps (n_q == 1)")
+    T, Hkv = k.shape[1], k.shape[2]
+    K = ids.shape[-1]
+    if out is None:
+        out = torch.empty((Bt, 1, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((Bt, 1, Hq), dtype=torch.float32, device=q.device)
+    sp = 0
+    if status is not None:
+        _dev(status, torch.int32, "status")
+        sp = status.data_ptr()
+    lib = load_library()
+    _check("msa_sparse_attn_decode_noalloc",
+           lib.msa_sparse_attn_decode_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                              ids.data_ptr(), out.data_ptr(), lse.data_ptr(), Bt,
+                                              T, Hq, Hkv, d, block, K, sp or None,
+                                              _stream(stream)))
     return out, lse
 
 

@@ -158,6 +158,41 @@ MSA_API msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *
                                       const msa_stage_events *events);
 
 /*
+ * Decode attention that allocates nothing.  The pages have no counterpart:
+ * this entry point is an addition of this library for callers that cannot
+ * allocate device memory or hand over a workspace -- for example a serving
+ * engine or plugin host that has already given all device memory to its own
+ * pool, where a cudaMalloc would fail or stall the whole device, and which
+ * has no spare buffer to pass as workspace.
+ *
+ * It computes exactly what msa_sparse_attn computes for a decode step (n_q = 1,
+ * same layouts, same split-K and combine kernels), but its scratch (the
+ * per-split partials) is a file-scope static __device__ array of
+ * MSA_NOALLOC_SCRATCH_BYTES (16 MiB).  That array is part of the library
+ * image: every GPU on which it has been loaded holds it until the process
+ * exits.  The caller still owns and passes every input and output.
+ *   - Limit: 256 + align256(Bt*K*S*Hq*d*4) + align256(Bt*K*S*Hq*4) bytes must
+ *     fit in the array, with S = ceil(block / 64); otherwise the call returns
+ *     MSA_ERR_WORKSPACE before enqueueing anything.  (The 4-sequence
+ *     1M-context decode, Bt 4, K 8, block 512, Hq 64, d 128, needs 8.5 MB.)
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture begins.
+ *   - Every call uses the same array, which keeps the contents of the last
+ *     call.  Calls whose kernels overlap on the GPU (two streams, or two host
+ *     threads) race on it and must be serialised by the caller.
+ *   - status: optional device int.  Kernels OR 2 into it when they skip an id
+ *     outside [-1, N).  With NULL those reports are dropped.
+ * No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define MSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+MSA_API msa_status msa_sparse_attn_decode_noalloc(const void *q, const void *k, const void *v,
+                                                  const int32_t *ids, float *out, float *lse,
+                                                  int Bt, int T, int Hq, int Hkv, int d,
+                                                  int block, int K, int *status, void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears the sticky device status word
  * of `workspace`: MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_BAD_IDS (the first found,
  * in that order of precedence: timeout first), or MSA_ERR_CUDA if the
