@@ -31,7 +31,8 @@ cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts
 // tcgen05 kernels (kernels_tc.cu)
 size_t selftest_smem_bytes(int N, int Kd);
 cudaError_t launch_selftest_umma(const CUtensorMap &tm_a, const CUtensorMap &tm_b, float *C,
-                                 int N, int Kd, int b_mn_major, int *status, cudaStream_t st);
+                                 int N, int Kd, int b_mn_major, int a_tmem, int *status,
+                                 cudaStream_t st);
 size_t prefill_index_smem_bytes(int d_idx);
 cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                  int32_t *ids, int *status, int num_sms, cudaStream_t st);

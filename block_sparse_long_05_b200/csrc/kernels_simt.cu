@@ -290,56 +290,83 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
 }
 
 // ------------------------------------------------------------------------
-// Log-sum-exp combine: one warp per (query row, head); P = K*S partials,
-// slot s valid when ids[row][s] >= 0 and the partial's lse is finite.
+// Log-sum-exp combine.  One CTA per (query row, group of HG heads).  The P =
+// K*S partials of each head are merged as LSE = log sum_p exp(lse_p) and
+// out = sum_p exp(lse_p - LSE) o_p.  Weights are computed once into shared
+// memory; the partial rows are then streamed with 16-byte loads (several in
+// flight per thread).  Partial p = (slot s, split sp) is valid when
+// ids[row][s] >= 0 and its lse is finite; invalid partials are never used
+// (their memory may hold a previous call's data).
 // ------------------------------------------------------------------------
 template <typename PT, int D>
 __global__ void __launch_bounds__(256) lse_combine_kernel(
     const PT *__restrict__ part_o, const float *__restrict__ part_lse,
-    const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out,
-    long long rows, int Hq, int K, int S) {
-    constexpr int PER = D / 32;  // elements per lane
-    const long long w = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
-    const int lane = threadIdx.x % 32;
-    if (w >= rows * Hq) return;
-    const long long row = w / Hq;
-    const int h = static_cast<int>(w % Hq);
-    float mx = -INFINITY;
-    for (int s = 0; s < K; ++s) {
-        if (ids[row * K + s] < 0) continue;
-        for (int p = 0; p < S; ++p) mx = fmaxf(mx, part_lse[((row * K + s) * S + p) * Hq + h]);
+    const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
+    int K, int S, int HG) {
+    constexpr int VEC = 16 / sizeof(PT);  // elements per 16-byte load
+    constexpr int NV = D / VEC;           // 16-byte loads per head row
+    extern __shared__ float wsm[];        // [P][HG] weights, then [HG] LSE
+    const long long row = blockIdx.x;
+    const int h0 = blockIdx.y * HG;
+    const int P = K * S;
+    float *Lsm = wsm + P * HG;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < P * HG; e += blockDim.x) {
+        const int pp = e / HG, hh = e % HG;
+        const int s = pp / S;
+        float l = -INFINITY;
+        if (ids[row * K + s] >= 0) l = part_lse[((row * K + s) * S + pp % S) * Hq + h0 + hh];
+        wsm[e] = l;
     }
-    float acc[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-    float L = -INFINITY;
-    if (mx != -INFINITY) {
-        float sum = 0.f;
-        for (int s = 0; s < K; ++s) {
-            if (ids[row * K + s] < 0) continue;
-            for (int p = 0; p < S; ++p) {
-                const float l = part_lse[((row * K + s) * S + p) * Hq + h];
+    __syncthreads();
+    for (int hh = tid; hh < HG; hh += blockDim.x) {
+        float mx = -INFINITY;
+        for (int pp = 0; pp < P; ++pp) mx = fmaxf(mx, wsm[pp * HG + hh]);
+        float L = -INFINITY;
+        if (mx != -INFINITY) {
+            float sum = 0.f;
+            for (int pp = 0; pp < P; ++pp) {
+                const float l = wsm[pp * HG + hh];
                 if (l != -INFINITY) sum += exp2f((l - mx) * kLog2e);
             }
+            L = mx + log2f(sum) * kLn2;
         }
-        L = mx + log2f(sum) * kLn2;
-        for (int s = 0; s < K; ++s) {
-            if (ids[row * K + s] < 0) continue;
-            for (int p = 0; p < S; ++p) {
-                const long long pr = (row * K + s) * S + p;
-                const float l = part_lse[pr * Hq + h];
-                if (l == -INFINITY) continue;
-                const float wgt = exp2f((l - L) * kLog2e);
-                const PT *src = part_o + (pr * Hq + h) * D + lane * PER;
+        for (int pp = 0; pp < P; ++pp) {
+            const float l = wsm[pp * HG + hh];
+            wsm[pp * HG + hh] = (l == -INFINITY) ? 0.f : exp2f((l - L) * kLog2e);
+        }
+        Lsm[hh] = L;
+        lse_out[row * Hq + h0 + hh] = L;
+    }
+    __syncthreads();
+    for (int e = tid; e < HG * NV; e += blockDim.x) {
+        const int hh = e / NV, c = (e % NV) * VEC;
+        float acc[VEC];
 #pragma unroll
-                for (int e = 0; e < PER; ++e) acc[e] = fmaf(wgt, static_cast<float>(src[e]), acc[e]);
+        for (int x = 0; x < VEC; ++x) acc[x] = 0.f;
+        const PT *src = part_o + ((row * K) * S * Hq + h0 + hh) * static_cast<long long>(D) + c;
+        const long long pstride = static_cast<long long>(Hq) * D;  // between consecutive partials
+#pragma unroll 4
+        for (int pp = 0; pp < P; ++pp) {
+            const float wgt = wsm[pp * HG + hh];
+            const uint4 u = *reinterpret_cast<const uint4 *>(src + pp * pstride);
+            if (sizeof(PT) == 2) {
+                float f[8];
+                bf16x8_to_f32(u, f);
+#pragma unroll
+                for (int x = 0; x < VEC; ++x) acc[x] += wgt != 0.f ? wgt * f[x] : 0.f;
+            } else {
+                const float f[4] = {__uint_as_float(u.x), __uint_as_float(u.y),
+                                    __uint_as_float(u.z), __uint_as_float(u.w)};
+#pragma unroll
+                for (int x = 0; x < VEC; ++x) acc[x] += wgt != 0.f ? wgt * f[x] : 0.f;
             }
         }
-    }
-    float *dst = out + (row * Hq + h) * D + lane * PER;
+        float *dst = out + (row * Hq + h0 + hh) * static_cast<long long>(D) + c;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) dst[e] = acc[e];
-    if (lane == 0) lse_out[row * Hq + h] = L;
+        for (int x = 0; x < VEC; x += 4)
+            *reinterpret_cast<float4 *>(dst + x) = make_float4(acc[x], acc[x + 1], acc[x + 2], acc[x + 3]);
+    }
 }
 
 // ------------------------------------------------------------------------
@@ -608,25 +635,29 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            const float *part_lse, const int32_t *ids, float *out, float *lse,
                            int S, cudaStream_t st) {
     const long long rows = static_cast<long long>(sh.Bt) * sh.n_q;
-    const long long warps = rows * sh.Hq;
-    const long long blocks = (warps + 7) / 8;
+    // heads per CTA: all of them when there are many rows, else fewer so the
+    // grid still covers the SMs a few times
+    int HG = sh.Hq;
+    while (HG > 1 && HG % 2 == 0 && rows * (sh.Hq / HG) < 1024) HG /= 2;
+    const int vec = part_bf16 ? 8 : 4;
+    int threads = HG * sh.d / vec;
+    threads = threads > 256 ? 256 : ((threads + 31) / 32) * 32;
+    const int P = sh.K * S;
+    const size_t smem = static_cast<size_t>(P * HG + HG) * sizeof(float);
+    const dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>(sh.Hq / HG));
+#define MSA_COMBINE(PT, DD)                                                                      \
+    do {                                                                                         \
+        cudaFuncSetAttribute(lse_combine_kernel<PT, DD>,                                         \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
+        lse_combine_kernel<PT, DD><<<grid, threads, smem, st>>>(                                 \
+            static_cast<const PT *>(part_o), part_lse, ids, out, lse, sh.Hq, sh.K, S, HG);       \
+    } while (0)
     if (part_bf16) {
-        const auto *po = static_cast<const __nv_bfloat16 *>(part_o);
-        if (sh.d == 128)
-            lse_combine_kernel<__nv_bfloat16, 128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-                po, part_lse, ids, out, lse, rows, sh.Hq, sh.K, S);
-        else
-            lse_combine_kernel<__nv_bfloat16, 64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-                po, part_lse, ids, out, lse, rows, sh.Hq, sh.K, S);
+        if (sh.d == 128) MSA_COMBINE(__nv_bfloat16, 128); else MSA_COMBINE(__nv_bfloat16, 64);
     } else {
-        const auto *po = static_cast<const float *>(part_o);
-        if (sh.d == 128)
-            lse_combine_kernel<float, 128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-                po, part_lse, ids, out, lse, rows, sh.Hq, sh.K, S);
-        else
-            lse_combine_kernel<float, 64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-                po, part_lse, ids, out, lse, rows, sh.Hq, sh.K, S);
+        if (sh.d == 128) MSA_COMBINE(float, 128); else MSA_COMBINE(float, 64);
     }
+#undef MSA_COMBINE
     return cudaGetLastError();
 }
 

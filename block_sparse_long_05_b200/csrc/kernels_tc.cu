@@ -59,7 +59,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ===========================================================================
 __global__ void __launch_bounds__(128, 1) selftest_umma_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-    float *__restrict__ C, int N, int Kd, int b_mn_major, int *status) {
+    float *__restrict__ C, int N, int Kd, int b_mn_major, int a_tmem_cols, int *status) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = align1024(smem_raw);
     unsigned char *a_s = base;                                  // Kd/64 regions x 16 KB
@@ -70,7 +70,9 @@ __global__ void __launch_bounds__(128, 1) selftest_umma_kernel(
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid / 32;
-    const uint32_t ncols = N <= 64 ? 64u : (N <= 128 ? 128u : 256u);
+    // accumulator columns [0, N); with A in tensor memory, A at [N, N + Kd/2)
+    const int need = N + (a_tmem_cols ? Kd / 2 : 0);
+    const uint32_t ncols = need <= 64 ? 64u : (need <= 128 ? 128u : (need <= 256 ? 256u : 512u));
     if (tid == 0) {
         mbar_init(bar_ld, 1);
         mbar_init(bar_mma, 1);
@@ -101,6 +103,29 @@ __global__ void __launch_bounds__(128, 1) selftest_umma_kernel(
         }
     }
     bool ok = mbar_wait(bar_ld, 0, abort_flag, status);
+    if (ok && a_tmem_cols) {
+        // A operand from tensor memory: each thread copies its row of A from
+        // the swizzled shared tile into TMEM columns [N, N + Kd/2), packed
+        // two bf16 per column, even k in the low half.
+        const int row = tid;
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        for (int c0 = 0; c0 < Kd; c0 += 32) {  // 32 elements = 16 columns per store
+            uint32_t w[16];
+            for (int q = 0; q < 4; ++q) {  // four 16-byte pieces of 8 elements
+                const int k = c0 + q * 8;
+                const uint4 u = *reinterpret_cast<const uint4 *>(
+                    a_s + (k / 64) * kRegionBytes + sw128_offset(row, (k % 64) / 8));
+                w[q * 4 + 0] = u.x;
+                w[q * 4 + 1] = u.y;
+                w[q * 4 + 2] = u.z;
+                w[q * 4 + 3] = u.w;
+            }
+            tmem_st16(tmem + lane_base + N + c0 / 2, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+    }
+    __syncthreads();
     if (ok && tid == 0) {
         tc_fence_after();
         const uint32_t idesc = idesc_bf16_f32(128, N, b_mn_major != 0);
@@ -111,7 +136,10 @@ __global__ void __launch_bounds__(128, 1) selftest_umma_kernel(
                 bd = sdesc_sw128(smem_addr(b_s + kk * 16 * 128), static_cast<uint32_t>(Kd) * 128, 1024);
             else
                 bd = sdesc_sw128(smem_addr(b_s + static_cast<size_t>(kk / 4) * N * 128 + (kk % 4) * 32), 16, 1024);
-            umma_bf16(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            if (a_tmem_cols)
+                umma_bf16_tmem_a(tmem, tmem + N + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
+            else
+                umma_bf16(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_mma);
     }
@@ -362,6 +390,24 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
 
 // ===========================================================================
 // Prefill attention (KV-block-outer).
+//
+// One CTA per SM, 256 threads = two warpgroups (WG0 = warps 0-3, WG1 = warps
+// 4-7).  A work item is (kv head hk, sequence b, block j, slice of the block's
+// hit list).  Thread 0 TMA-loads K_j and V_j of head hk into shared memory
+// once per item (block <= 128) or per 128-key sub-tile (block > 128).  The
+// item's hit list is cut into 128-row chunks (128/G tokens x G heads); the
+// two warpgroups take alternate chunks and run them independently, so one
+// warpgroup's softmax overlaps the other's tensor-core work:
+//   gather Q rows (cp.async, double-buffered per warpgroup)
+//   S = Q K^T          (tcgen05, S in tensor memory)
+//   P = exp2(S*c - m)  (registers; P written back over S as bf16)
+//   O = P V            (tcgen05, A operand read from tensor memory)
+//   partial row: O / l in bf16, lse = ln(l) + m  (per query, slot and head)
+// Tensor memory: WG w owns columns [256w, 256w+256): S/P at +0, O at +128.
+// With block > 128 the warpgroups walk the sub-tiles in lockstep (K/V
+// double-buffered) with an online softmax; the O rescale is only done when
+// the running max grows by more than 2^8, which keeps P <= 256 and the
+// result exact up to rounding.
 // ===========================================================================
 struct AttnParams {
     const __nv_bfloat16 *q;
@@ -373,72 +419,86 @@ struct AttnParams {
     float *part_lse;
     int *status;
     int Bt, n_q, T, Hq, Hkv, G, block, K, N;
-    int NK;   // keys per sub-tile (min(block, 128))
-    int NS;   // sub-tiles per block
-    int TOK;  // tokens per 128-row chunk = 128 / G
+    int NK;      // keys per sub-tile (min(block, 128))
+    int NS;      // sub-tiles per block
+    int TOK;     // tokens per 128-row chunk = 128 / G
+    int log2G;
     float scale_log2;
 };
 
+// Per-chunk token table, filled by the gathering warpgroup.
+struct ChunkRows {
+    long long qoff[128];  // element offset of the token's first head of group hk in q
+    int entry[128];       // list entry = partial row (b*n_q + i)*K + slot, or -1
+    int t[128];           // query position, or -1
+};
+
 template <int D>
-__global__ void __launch_bounds__(128, 1) prefill_attn_kernel(
+__global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     AttnParams p) {
     constexpr int DREG = D / 64;                 // swizzled regions per Q row block
     constexpr uint32_t QBYTES = DREG * kRegionBytes;
+    constexpr int PPR = D / 8;                   // 16-byte pieces per Q row
     const int NK = p.NK;
     const uint32_t kv_tile = static_cast<uint32_t>(NK) * 128u * DREG;  // one of K or V
-    const int KVST = p.NS > 1 ? 2 : 1;
+    const bool streamed = p.NS > 1;
+    const int KVST = streamed ? 2 : 1;
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = align1024(smem_raw);
     unsigned char *kv_s = base;                                   // KVST x (K tile, V tile)
-    unsigned char *q_s = kv_s + KVST * 2 * kv_tile;               // 2 x QBYTES
-    unsigned char *p_s = q_s + 2 * QBYTES;                        // NK/64 regions
-    unsigned char *tail = p_s + ((NK + 63) / 64) * kRegionBytes;
-    uint64_t *kvfull = reinterpret_cast<uint64_t *>(tail);        // [2]
-    uint64_t *bar_s = kvfull + 2;
-    uint64_t *bar_o = kvfull + 3;
-    int *tok_entry = reinterpret_cast<int *>(kvfull + 4);         // [2][128]
-    int *sh_item = tok_entry + 256;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sh_item + 1);
+    unsigned char *q_s = kv_s + KVST * 2 * kv_tile;               // [wg][buf] Q tiles
+    const int QBUF = streamed ? 1 : 2;
+    unsigned char *tail = q_s + 2 * QBUF * QBYTES;
+    ChunkRows *rows_s = reinterpret_cast<ChunkRows *>(tail);      // [wg][buf]
+    uint64_t *kvfull = reinterpret_cast<uint64_t *>(rows_s + 2 * QBUF);  // [2]
+    uint64_t *bar_s = kvfull + 2;                                 // [wg]
+    uint64_t *bar_o = kvfull + 4;                                 // [wg]
+    int *sh_item = reinterpret_cast<int *>(kvfull + 6);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sh_item + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid / 32;
+    const int wg = tid >> 7, wtid = tid & 127;
+    const uint32_t wg_bar = 1 + wg;  // named barrier per warpgroup
     if (tid == 0) {
         mbar_init(kvfull, 1);
         mbar_init(kvfull + 1, 1);
         mbar_init(bar_s, 1);
+        mbar_init(bar_s + 1, 1);
         mbar_init(bar_o, 1);
+        mbar_init(bar_o + 1, 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_s = tmem;        // S: columns [0, NK)
-    const uint32_t tmem_o = tmem + 128;  // O: columns [128, 128 + D)
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tmem = *tmem_slot + static_cast<uint32_t>(wg * 256);
+    const uint32_t tmem_s = tmem;        // S (fp32) / P (bf16 pairs)
+    const uint32_t tmem_o = tmem + 128;  // O (fp32)
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
 
     const int n_items = p.counters[0];
     const int total = n_items * p.Hkv;
     const int G = p.G, TOK = p.TOK, K = p.K;
     const uint32_t idesc_s = idesc_bf16_f32(128, NK, false);
     const uint32_t idesc_o = idesc_bf16_f32(128, D, true);
-    const int row = tid;  // M row of this thread (TMEM lane)
-    const int tok = row / G, g = row % G;
+    const int row = wtid;                // M row = TMEM lane of this thread
+    const int tok = row >> p.log2G, g = row & (G - 1);
 
-    uint32_t kv_issue = 0, kv_use = 0, s_n = 0, o_n = 0;
+    uint32_t kv_issue = 0, kv_use = 0, s_n = 0, o_n = 0, item_n = 0;
     int armed_parity[2] = {-1, -1};
     bool aborted = false;
 
-    // Issue the K/V loads of sub-tile kt of block (b, j), kv head hk.
+    // K/V loads of sub-tile kt of block (b, j), kv head hk (thread 0 only).
     auto issue_kv = [&](int b, int j, int hk, int kt) {
         const uint32_t st = kv_issue % KVST;
         unsigned char *kd = kv_s + st * 2 * kv_tile;
@@ -453,34 +513,40 @@ __global__ void __launch_bounds__(128, 1) prefill_attn_kernel(
         ++kv_issue;
     };
 
-    // Gather the G heads of the chunk's tokens into Q buffer qb (cp.async).
-    auto gather_q = [&](int qb, int hk, int b, int list_base, int chunk, int ntok_item) {
-        unsigned char *dst_base = q_s + qb * QBYTES;
-        const int tok0 = chunk * TOK;
-        if (tid < TOK) {
-            int e = -1;
-            if (tok0 + tid < ntok_item) {
-                e = p.entries[list_base + tok0 + tid];
-                const long long qrow = e / K;
-                if (e < 0 || qrow >= static_cast<long long>(p.Bt) * p.n_q || qrow / p.n_q != b) {
+    // Token table of chunk `c` into rows_s[wg][buf], then the cp.async gather
+    // of its 128 Q rows into q_s[wg][buf].  Called by one whole warpgroup.
+    auto gather = [&](int buf, int hk, int b, int list_base, int c, int ntok) {
+        ChunkRows &cr = rows_s[wg * QBUF + buf];
+        const int tok0 = c * TOK;
+        if (wtid < TOK) {
+            int e = -1, t = -1;
+            long long qoff = 0;
+            if (tok0 + wtid < ntok) {
+                e = p.entries[list_base + tok0 + wtid];
+                const int qrow = e >= 0 ? e / K : -1;
+                const int bi = qrow >= 0 ? qrow / p.n_q : -1;
+                if (e < 0 || bi != b) {
                     atomicOr(p.status, kDevBadIds);
                     e = -1;
+                } else {
+                    t = p.T - p.n_q + (qrow - bi * p.n_q);
+                    qoff = (static_cast<long long>(qrow) * p.Hq + static_cast<long long>(hk) * G) * D;
                 }
             }
-            tok_entry[qb * 128 + tid] = e;
+            cr.entry[wtid] = e;
+            cr.t[wtid] = t;
+            cr.qoff[wtid] = qoff;
         }
-        constexpr int PPR = D / 8;  // 16-byte pieces per row
-        for (int pc = tid; pc < 128 * PPR; pc += 128) {
+        named_barrier(wg_bar, 128);
+        unsigned char *dst_base = q_s + (wg * QBUF + buf) * QBYTES;
+#pragma unroll 4
+        for (int pc = wtid; pc < 128 * PPR; pc += 128) {
             const int r = pc / PPR, cc = pc % PPR;
-            const int tk = r / G, gg = r % G;
-            int e = -1;
-            if (tok0 + tk < ntok_item) e = p.entries[list_base + tok0 + tk];
-            const long long qrow = e / K;
-            const bool ok = e >= 0 && qrow < static_cast<long long>(p.Bt) * p.n_q && qrow / p.n_q == b;
-            const __nv_bfloat16 *src =
-                ok ? p.q + ((qrow * p.Hq + hk * G + gg) * D + cc * 8) : p.q;
-            unsigned char *dst = dst_base + (cc / 8) * kRegionBytes + sw128_offset(r, cc % 8);
-            cp_async_16(dst, src, ok ? 16u : 0u);
+            const int tk = r >> p.log2G, gg = r & (G - 1);
+            const bool ok = cr.t[tk] >= 0;
+            const __nv_bfloat16 *src = p.q + (ok ? cr.qoff[tk] + gg * D + cc * 8 : 0);
+            cp_async_16(dst_base + (cc / 8) * kRegionBytes + sw128_offset(r, cc % 8), src,
+                        ok ? 16u : 0u);
         }
         cp_async_commit();
     };
@@ -489,146 +555,176 @@ __global__ void __launch_bounds__(128, 1) prefill_attn_kernel(
         if (tid == 0) *sh_item = atomicAdd(p.counters + 1, 1);
         __syncthreads();
         const int w = *sh_item;
-        if (w >= total) break;
+        if (w >= total || *abort_flag) break;
         const int hk = w / n_items;
-        const AttnItem item = p.items[w % n_items];
-        const int b = item.pair / p.N, j = item.pair % p.N;
+        const AttnItem item = p.items[w - hk * n_items];
+        const int b = item.pair / p.N, j = item.pair - b * p.N;
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
-        const int n_steps = n_chunks * p.NS;
+        // chunks of this warpgroup: c = wg, wg + 2, ...
+        const int my_chunks = n_chunks > wg ? (n_chunks - wg + 1) / 2 : 0;
+        // steps: with streamed K/V both warpgroups walk (chunk pair, sub-tile)
+        // in lockstep, otherwise each walks its own chunks
+        const int pairs = (n_chunks + 1) / 2;
+        const int n_steps = streamed ? pairs * p.NS : my_chunks;
 
         if (tid == 0) issue_kv(b, j, hk, 0);
-        gather_q(0, hk, b, list_base, 0, ntok);
+        if (my_chunks > 0) gather(0, hk, b, list_base, wg, ntok);
 
         float m_run = -INFINITY, l_run = 0.f;
         for (int step = 0; step < n_steps; ++step) {
-            const int c = step / p.NS, kt = step % p.NS;
-            const int qb = c & 1;
+            const int ci = streamed ? step / p.NS : step;   // index among my chunks
+            const int kt = streamed ? step % p.NS : 0;
+            const int c = wg + 2 * ci;                      // chunk index in the item
+            const bool active = c < n_chunks;
+            const int buf = streamed ? 0 : (ci & 1);
+            // ---- Q of this chunk: gathered at item start (first chunk), by the
+            // previous step's prefetch, or here (streamed: single Q buffer)
+            if (streamed && kt == 0 && ci > 0 && active) gather(0, hk, b, list_base, c, ntok);
             if (kt == 0) cp_async_wait_all();
             fence_proxy_async_smem();
-            __syncthreads();
-            // wait for this step's K/V tile
-            const uint32_t st = kv_use % KVST;
             bool ok = true;
-            if (p.NS > 1 || c == 0) {
+            uint32_t st = 0;
+            if (streamed) {
+                // lockstep: both warpgroups use this sub-tile; the other stage
+                // is free once both finished their PV of the previous step
+                st = kv_use % KVST;
                 ok = mbar_wait(kvfull + st, (kv_use / KVST) & 1, abort_flag, p.status);
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
                 ++kv_use;
-                armed_parity[st] = -1;
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+                if (tid == 0 && step + 1 < n_steps) issue_kv(b, j, hk, (step + 1) % p.NS);
+            } else {
+                // one K/V load per item (stage 0), the item_n-th of this CTA
+                if (step == 0) ok = mbar_wait(kvfull, item_n & 1, abort_flag, p.status);
+                if (named_barrier_or(wg_bar, 128, !ok || *abort_flag)) { aborted = true; break; }
             }
             unsigned char *kd = kv_s + st * 2 * kv_tile;
             unsigned char *vd = kd + kv_tile;
-            if (tid == 0) {
+            if (active && wtid == 0) {
                 tc_fence_after();
-                const uint32_t qa = smem_addr(q_s + qb * QBYTES), ka = smem_addr(kd);
+                const uint32_t qa = smem_addr(q_s + (wg * QBUF + buf) * QBYTES), ka = smem_addr(kd);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < D / 16; ++kk)
                     umma_bf16(tmem_s,
                               sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
                               sdesc_sw128(ka + (kk / 4) * NK * 128 + (kk % 4) * 32, 16, 1024),
                               idesc_s, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(bar_s);
-                // prefetch the next sub-tile of this block (streamed K/V)
-                if (p.NS > 1 && step + 1 < n_steps) issue_kv(b, j, hk, (step + 1) % p.NS);
+                umma_commit(bar_s + wg);
             }
-            if (kt == 0 && c + 1 < n_chunks) gather_q(qb ^ 1, hk, b, list_base, c + 1, ntok);
-            ok = mbar_wait(bar_s, s_n & 1, abort_flag, p.status);
-            ++s_n;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-            tc_fence_after();
-
-            // ---- softmax for row `row`
-            const int e = tok_entry[qb * 128 + tok];
-            const bool valid = e >= 0;
-            const long long qrow = valid ? e / K : 0;
-            const int t = p.T - p.n_q + static_cast<int>(qrow % p.n_q);
-            const int kbase = j * p.block + kt * NK;
-            const int lim = valid ? t - kbase : -1;  // valid columns: col <= lim
-            float mt = -INFINITY;
-            for (int cc = 0; cc < NK / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld32(tmem_s + lane_addr + cc * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int x = 0; x < 32; ++x)
-                    if (cc * 32 + x <= lim) mt = fmaxf(mt, __uint_as_float(v[x]));
+            // prefetch the next chunk's Q while this one computes
+            if (!streamed && ci + 1 < my_chunks) gather(buf ^ 1, hk, b, list_base, c + 2, ntok);
+            if (active) {
+                ok = mbar_wait(bar_s + wg, s_n & 1, abort_flag, p.status);
+                ++s_n;
             }
-            mt *= p.scale_log2;
-            if (kt == 0) {
-                m_run = mt;
-                l_run = 0.f;
+            if (streamed) {
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
             } else {
-                float alpha = 1.f;
-                bool need = false;
-                if (mt > m_run + 8.f) {
-                    alpha = exp2f(m_run - mt);
-                    m_run = mt;
-                    l_run *= alpha;
-                    need = true;
-                }
-                if (__any_sync(0xFFFFFFFFu, need)) {
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem_o + lane_addr + cc * 32, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
-                        tmem_st32(tmem_o + lane_addr + cc * 32, v);
-                    }
-                    tmem_wait_st();
-                }
+                if (named_barrier_or(wg_bar, 128, !ok || *abort_flag)) { aborted = true; break; }
             }
-            unsigned char *prow_base = p_s;
-            for (int cc = 0; cc < NK / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld32(tmem_s + lane_addr + cc * 32, v);
-                tmem_wait_ld();
-                float pv[32];
-#pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    const bool in = cc * 32 + x <= lim;
-                    pv[x] = in ? exp2f(__uint_as_float(v[x]) * p.scale_log2 - m_run) : 0.f;
-                    l_run += pv[x];
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int col = cc * 32 + q4 * 8;  // first key of this 16-byte piece
-                    uint4 u;
-                    u.x = pack_bf16x2(pv[q4 * 8 + 0], pv[q4 * 8 + 1]);
-                    u.y = pack_bf16x2(pv[q4 * 8 + 2], pv[q4 * 8 + 3]);
-                    u.z = pack_bf16x2(pv[q4 * 8 + 4], pv[q4 * 8 + 5]);
-                    u.w = pack_bf16x2(pv[q4 * 8 + 6], pv[q4 * 8 + 7]);
-                    *reinterpret_cast<uint4 *>(prow_base + (col / 64) * kRegionBytes +
-                                               sw128_offset(row, (col % 64) / 8)) = u;
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (tid == 0) {
+            if (active) {
                 tc_fence_after();
-                const uint32_t pa = smem_addr(p_s), va = smem_addr(vd);
-                for (int kk = 0; kk < NK / 16; ++kk) {
-                    umma_bf16(tmem_o,
-                              sdesc_sw128(pa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
-                              sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
-                              idesc_o, (kt > 0 || kk > 0) ? 1u : 0u);
+                const ChunkRows &cr = rows_s[wg * QBUF + buf];
+                const int t = cr.t[tok];
+                const int lim = t - (j * p.block + kt * NK);  // valid key columns: <= lim
+                // ---- softmax of this row (registers)
+                float sv[128];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    if (cc * 32 < NK) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem_s + lane_addr + cc * 32, v);
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) sv[cc * 32 + x] = __uint_as_float(v[x]);
+                    }
                 }
-                umma_commit(bar_o);
+                tmem_wait_ld();
+                if (lim < NK - 1) {
+#pragma unroll
+                    for (int x = 0; x < 128; ++x)
+                        if (x > lim) sv[x] = -INFINITY;
+                }
+                float mt = -INFINITY;
+#pragma unroll
+                for (int x = 0; x < 128; ++x)
+                    if (x < NK) mt = fmaxf(mt, sv[x]);
+                mt *= p.scale_log2;
+                if (kt == 0) {
+                    m_run = mt;
+                    l_run = 0.f;
+                } else {
+                    float alpha = 1.f;
+                    bool need = false;
+                    if (mt > m_run + 8.f) {
+                        alpha = ex2_approx(m_run - mt);
+                        m_run = mt;
+                        l_run *= alpha;
+                        need = true;
+                    }
+                    if (__any_sync(0xFFFFFFFFu, need)) {
+                        for (int cc = 0; cc < D / 32; ++cc) {
+                            uint32_t v[32];
+                            tmem_ld32(tmem_o + lane_addr + cc * 32, v);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int x = 0; x < 32; ++x)
+                                v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
+                            tmem_st32(tmem_o + lane_addr + cc * 32, v);
+                        }
+                        tmem_wait_st();
+                    }
+                }
+                const float mref = m_run == -INFINITY ? 0.f : m_run;
+                float lsum = 0.f;
+#pragma unroll
+                for (int g32 = 0; g32 < 4; ++g32) {  // 32 keys -> 16 packed columns
+                    if (g32 * 32 < NK) {
+                        uint32_t w16[16];
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            const float p0 = ex2_approx(fmaf(sv[g32 * 32 + 2 * x], p.scale_log2, -mref));
+                            const float p1 = ex2_approx(fmaf(sv[g32 * 32 + 2 * x + 1], p.scale_log2, -mref));
+                            lsum += p0 + p1;
+                            w16[x] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st16(tmem_s + lane_addr + g32 * 16, w16);
+                    }
+                }
+                l_run += lsum;
+                tmem_wait_st();
+                tc_fence_before();
             }
-            ok = mbar_wait(bar_o, o_n & 1, abort_flag, p.status);
-            ++o_n;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-            tc_fence_after();
-
-            if (kt == p.NS - 1) {
-                // ---- epilogue: normalised partial and its lse
-                const int slot = valid ? static_cast<int>(e % K) : 0;
+            named_barrier(wg_bar, 128);
+            if (active && wtid == 0) {
+                tc_fence_after();
+                const uint32_t va = smem_addr(vd);
+                for (int kk = 0; kk < NK / 16; ++kk)
+                    umma_bf16_tmem_a(tmem_o, tmem_s + kk * 8,
+                                     sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
+                                     idesc_o, (kt > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(bar_o + wg);
+            }
+            if (active) {
+                ok = mbar_wait(bar_o + wg, o_n & 1, abort_flag, p.status);
+                ++o_n;
+            }
+            if (streamed) {
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+            } else {
+                if (named_barrier_or(wg_bar, 128, !ok || *abort_flag)) { aborted = true; break; }
+            }
+            if (active && kt == p.NS - 1) {
+                tc_fence_after();
+                // ---- epilogue: normalised bf16 partial and its lse
+                const ChunkRows &cr = rows_s[wg * QBUF + buf];
+                const int e = cr.entry[tok];
+                const bool valid = e >= 0;
                 const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-                __nv_bfloat16 *dst =
-                    p.part_o + ((qrow * K + slot) * p.Hq + static_cast<long long>(hk) * G + g) * D;
+                const long long prow = static_cast<long long>(valid ? e : 0) * p.Hq +
+                                       static_cast<long long>(hk) * G + g;
+                __nv_bfloat16 *dst = p.part_o + prow * D;
+#pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t v[32];
                     tmem_ld32(tmem_o + lane_addr + cc * 32, v);
@@ -646,24 +742,28 @@ __global__ void __launch_bounds__(128, 1) prefill_attn_kernel(
                     }
                 }
                 if (valid)
-                    p.part_lse[(qrow * K + slot) * p.Hq + static_cast<long long>(hk) * G + g] =
-                        l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
+                    p.part_lse[prow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
                 m_run = -INFINITY;
                 l_run = 0.f;
+                tc_fence_before();
             }
-            tc_fence_before();
         }
-        if (aborted) break;
+        ++item_n;
+        // both warpgroups done with this item's K/V and Q buffers
+        if (__syncthreads_or(aborted)) {
+            aborted = true;
+            break;
+        }
     }
     __syncthreads();
     if (aborted && tid == 0) {
-        for (int s = 0; s < 2; ++s)
-            if (armed_parity[s] >= 0) mbar_drain(kvfull + s, static_cast<uint32_t>(armed_parity[s]));
+        for (int s2 = 0; s2 < 2; ++s2)
+            if (armed_parity[s2] >= 0) mbar_drain(kvfull + s2, static_cast<uint32_t>(armed_parity[s2]));
     }
     cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (warp == 0) tmem_dealloc(*tmem_slot, 512);
 }
 
 }  // namespace
@@ -674,11 +774,12 @@ size_t selftest_smem_bytes(int N, int Kd) {
 }
 
 cudaError_t launch_selftest_umma(const CUtensorMap &tm_a, const CUtensorMap &tm_b, float *C,
-                                 int N, int Kd, int b_mn_major, int *status, cudaStream_t st) {
+                                 int N, int Kd, int b_mn_major, int a_tmem, int *status,
+                                 cudaStream_t st) {
     const size_t smem = selftest_smem_bytes(N, Kd);
     cudaFuncSetAttribute(selftest_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
-    selftest_umma_kernel<<<1, 128, smem, st>>>(tm_a, tm_b, C, N, Kd, b_mn_major, status);
+    selftest_umma_kernel<<<1, 128, smem, st>>>(tm_a, tm_b, C, N, Kd, b_mn_major, a_tmem, status);
     return cudaGetLastError();
 }
 
@@ -723,10 +824,10 @@ size_t prefill_attn_smem_bytes(const Shape &sh) {
     const int NK = sh.block < 128 ? sh.block : 128;
     const int NS = sh.block / NK;
     const int KVST = NS > 1 ? 2 : 1;
+    const int QBUF = NS > 1 ? 1 : 2;
     const size_t kv_tile = static_cast<size_t>(NK) * 128 * (sh.d / 64);
     const size_t q = static_cast<size_t>(sh.d / 64) * kRegionBytes;
-    const size_t pb = static_cast<size_t>((NK + 63) / 64) * kRegionBytes;
-    return 1024 + KVST * 2 * kv_tile + 2 * q + pb + 64 + 256 * 4 + 32;
+    return 1024 + KVST * 2 * kv_tile + 2 * QBUF * q + 2 * QBUF * sizeof(ChunkRows) + 64 + 32;
 }
 
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
@@ -754,16 +855,18 @@ cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const 
     ap.NK = sh.block < 128 ? sh.block : 128;
     ap.NS = sh.block / ap.NK;
     ap.TOK = 128 / sh.G;
+    ap.log2G = 0;
+    while ((1 << ap.log2G) < sh.G) ++ap.log2G;
     ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(sh.d));
     const size_t smem = prefill_attn_smem_bytes(sh);
     if (sh.d == 128) {
         cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
-        prefill_attn_kernel<128><<<num_sms, 128, smem, st>>>(tm_k, tm_v, ap);
+        prefill_attn_kernel<128><<<num_sms, 256, smem, st>>>(tm_k, tm_v, ap);
     } else {
         cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
-        prefill_attn_kernel<64><<<num_sms, 128, smem, st>>>(tm_k, tm_v, ap);
+        prefill_attn_kernel<64><<<num_sms, 256, smem, st>>>(tm_k, tm_v, ap);
     }
     return cudaGetLastError();
 }

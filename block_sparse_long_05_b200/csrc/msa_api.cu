@@ -59,7 +59,7 @@ WsLayout layout_for(const Shape &sh, bool with_attn) {
     };
     const long long pairs = static_cast<long long>(sh.Bt) * sh.N;
     L.n_chunks = (sh.n_q + kInvRows - 1) / kInvRows;
-    L.rows_per_item = with_attn ? 4 * (128 / sh.G) : 128;
+    L.rows_per_item = with_attn ? 16 * (128 / sh.G) : 128;  // 16 chunks of 128 rows
     L.max_items = static_cast<int>((static_cast<long long>(sh.Bt) * sh.n_q * sh.K + L.rows_per_item - 1) /
                                        L.rows_per_item +
                                    pairs);
@@ -322,12 +322,13 @@ msa_status msa_selftest_umma(const void *A, const void *B, float *C, int N, int 
     if (!A || !B || !C || !status) return MSA_ERR_INVALID_ARG;
     if (!(N == 64 || N == 128 || N == 256) || Kd < 64 || Kd > 256 || Kd % 64 != 0)
         return MSA_ERR_UNSUPPORTED;
+    const int b_mn = b_mn_major & 1;
     CUtensorMap ta, tb;
     const cuuint64_t da[2] = {static_cast<cuuint64_t>(Kd), 128};
     const cuuint64_t sa[1] = {static_cast<cuuint64_t>(Kd) * 2};
     const cuuint32_t ba[2] = {64, 128};
     if (!make_tmap(&ta, A, 2, da, sa, ba)) return MSA_ERR_CUDA;
-    if (b_mn_major) {
+    if (b_mn) {
         const cuuint64_t db[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(Kd)};
         const cuuint64_t sb[1] = {static_cast<cuuint64_t>(N) * 2};
         const cuuint32_t bb[2] = {64, static_cast<cuuint32_t>(Kd)};
@@ -338,8 +339,8 @@ msa_status msa_selftest_umma(const void *A, const void *B, float *C, int N, int 
         const cuuint32_t bb[2] = {64, static_cast<cuuint32_t>(N)};
         if (!make_tmap(&tb, B, 2, db, sb, bb)) return MSA_ERR_CUDA;
     }
-    return cuda_status(launch_selftest_umma(ta, tb, C, N, Kd, b_mn_major, status,
-                                            static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_selftest_umma(ta, tb, C, N, Kd, b_mn_major & 1, (b_mn_major >> 1) & 1,
+                                            status, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -254,8 +254,10 @@ def status_string(code: int) -> str:
     return load_library().msa_status_string(int(code)).decode()
 
 
-def selftest_umma(A: torch.Tensor, B: torch.Tensor, b_mn_major: bool, stream=None):
-    """C[128, N] = A[128, Kd] @ B with B as [N, Kd] (K-major) or [Kd, N] (MN-major)."""
+def selftest_umma(A: torch.Tensor, B: torch.Tensor, b_mn_major: bool, a_tmem: bool = False,
+                  stream=None):
+    """C[128, N] = A[128, Kd] @ B with B as [N, Kd] (K-major) or [Kd, N] (MN-major);
+    a_tmem: the MMA reads A from tensor memory."""
     _dev(A, torch.bfloat16, "A")
     _dev(B, torch.bfloat16, "B")
     Kd = A.shape[1]
@@ -263,7 +265,8 @@ def selftest_umma(A: torch.Tensor, B: torch.Tensor, b_mn_major: bool, stream=Non
     C = torch.empty((128, N), dtype=torch.float32, device=A.device)
     status = torch.zeros(1, dtype=torch.int32, device=A.device)
     lib = load_library()
+    flags = int(b_mn_major) | (2 if a_tmem else 0)
     _check("msa_selftest_umma", lib.msa_selftest_umma(A.data_ptr(), B.data_ptr(), C.data_ptr(), N,
-                                                      Kd, int(b_mn_major), status.data_ptr(),
+                                                      Kd, flags, status.data_ptr(),
                                                       _stream(stream)))
     return C, status

@@ -205,9 +205,11 @@ MSA_API const char *msa_status_string(int status);
 
 /*
  * Tensor-core self-test, not part of the method: C[128][N] = A . B with
- * A [128][Kd] bf16 (K-major) and B either as [N][Kd] (b_mn_major = 0, K-major)
- * or as [Kd][N] (b_mn_major = 1), C fp32, through the same TMA, shared-memory
- * descriptor, tcgen05.mma and TMEM read-back code the attention kernels use.
+ * A [128][Kd] bf16 (K-major) and B either as [N][Kd] (bit 0 of b_mn_major = 0,
+ * K-major) or as [Kd][N] (bit 0 = 1), C fp32, through the same TMA,
+ * shared-memory descriptor, tcgen05.mma and TMEM read-back code the attention
+ * kernels use.  Bit 1 of b_mn_major set: A is first copied into tensor memory
+ * and the MMA reads it from there (the layout the attention kernel uses for P).
  * N in {64, 128, 256}, Kd a multiple of 64 up to 256.  Device pointers;
  * `status` is a device int the kernel sets non-zero on a wait timeout.
  */
