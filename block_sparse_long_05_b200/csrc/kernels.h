@@ -37,6 +37,7 @@ size_t prefill_index_smem_bytes(int d_idx);
 cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                  int32_t *ids, int *status, int num_sms, cudaStream_t st);
 size_t prefill_attn_smem_bytes(const Shape &sh);
+int prefill_attn_rows_per_item(int G);
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                 const void *q, const int32_t *row_ptr, const int32_t *entries,
                                 const AttnItem *items, int *counters, void *part_o,

@@ -50,103 +50,121 @@ __device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
 
 // ------------------------------------------------------------------------
 // Decode index scan: block_scores[b][j] = max_{i in block j} q_idx[b].k_idx[b][i]
-// for j < own = (T-1)/block.  One warp per (b, j); 16-byte streaming loads,
-// D_IDX/8 lanes per key row.  fp32 accumulation (exact for integer keys).
+// for j < own = (T-1)/block.  One CTA of 8 warps per (b, j); the warps split
+// the block's rows; D_IDX/8 lanes per key row with 16-byte streaming loads,
+// 16 loads in flight per warp.  fp32 accumulation (exact for integer keys).
 // ------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ld_stream16(const uint4 *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 template <int D_IDX>
 __global__ void __launch_bounds__(256) decode_index_scan_kernel(
     const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16 *__restrict__ k_idx,
-    float *__restrict__ block_scores, int Bt, int T, int block, int own, int N) {
+    float *__restrict__ block_scores, int T, int block, int own, int N) {
     constexpr int LPR = D_IDX / 8;  // lanes per key row
     constexpr int RPL = 32 / LPR;   // key rows per warp load
-    const int lane = threadIdx.x & 31;
-    const int sub = lane / LPR;
-    const int part = lane % LPR;
-    const long long warps_total = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
-    const long long work = static_cast<long long>(Bt) * own;
-    int cur_b = -1;
+    constexpr int UNR = 16;         // loads in flight per warp
+    __shared__ float wmax[8];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int sub = lane / LPR, part = lane % LPR;
+    const int b = blockIdx.x / own, j = blockIdx.x % own;
     float qv[8];
-    for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
-         w < work; w += warps_total) {
-        const int b = static_cast<int>(w / own);
-        const int j = static_cast<int>(w % own);
-        if (b != cur_b) {
-            const uint4 qu =
-                *reinterpret_cast<const uint4 *>(q_idx + static_cast<long long>(b) * D_IDX + part * 8);
-            bf16x8_to_f32(qu, qv);
-            cur_b = b;
+    bf16x8_to_f32(*reinterpret_cast<const uint4 *>(q_idx + static_cast<long long>(b) * D_IDX + part * 8), qv);
+    const uint4 *base = reinterpret_cast<const uint4 *>(
+        k_idx + (static_cast<long long>(b) * T + static_cast<long long>(j) * block) * D_IDX);
+    // rows of this warp: r = (warp + 8 * it) * RPL + sub
+    const int groups = block / RPL;  // row groups of RPL rows
+    float best = -FLT_MAX;
+    for (int g0 = warp; g0 < groups; g0 += 8 * UNR) {
+        uint4 ku[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int gi = g0 + 8 * u;
+            ku[u] = gi < groups ? ld_stream16(base + (gi * RPL + sub) * LPR + part) : make_uint4(0, 0, 0, 0);
         }
-        const uint4 *base = reinterpret_cast<const uint4 *>(
-            k_idx + (static_cast<long long>(b) * T + static_cast<long long>(j) * block) * D_IDX);
-        float best = -FLT_MAX;
-        const int iters = block / RPL;
-#pragma unroll 8
-        for (int it = 0; it < iters; ++it) {
-            const int r = sub + RPL * it;
-            const uint4 ku = __ldcs(base + r * LPR + part);
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
             float kf[8];
-            bf16x8_to_f32(ku, kf);
+            bf16x8_to_f32(ku[u], kf);
             float s = 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) s = fmaf(qv[e], kf[e], s);
 #pragma unroll
             for (int o = LPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-            best = fmaxf(best, s);
+            if (g0 + 8 * u < groups) best = fmaxf(best, s);
         }
+    }
 #pragma unroll
-        for (int o = LPR; o < 32; o <<= 1) best = fmaxf(best, __shfl_xor_sync(0xFFFFFFFFu, best, o));
-        if (lane == 0) block_scores[static_cast<long long>(b) * N + j] = best;
+    for (int o = LPR; o < 32; o <<= 1) best = fmaxf(best, __shfl_xor_sync(0xFFFFFFFFu, best, o));
+    if (lane == 0) wmax[warp] = best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = wmax[0];
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
+        block_scores[static_cast<long long>(b) * N + j] = m;
     }
 }
 
 // ------------------------------------------------------------------------
-// Decode select: one warp per sequence.  Each lane keeps a sorted top list of
-// its strided candidates, then min(K, own+1)-1 rounds of warp arg-max over
-// the lanes' heads pick the winners; own is added and ids written ascending.
+// Decode select: one CTA of 1024 threads per sequence.  Each thread keeps the
+// best of its strided candidates (key = score desc, block asc, packed in 64
+// bits); min(K, own+1)-1 rounds of block arg-max pick the winners (the owner
+// of a winner advances to its next best); own is added, ids written ascending.
 // ------------------------------------------------------------------------
-template <int CAP>
-__global__ void __launch_bounds__(32) decode_select_kernel(const float *__restrict__ block_scores,
-                                                           int32_t *__restrict__ ids, int N,
-                                                           int own, int K) {
+constexpr int kSelThreads = 1024;
+
+__global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
+    const float *__restrict__ block_scores, int32_t *__restrict__ ids, int N, int own, int K) {
     const int b = blockIdx.x;
-    const int lane = threadIdx.x;
-    uint64_t top[CAP];
-#pragma unroll
-    for (int p = 0; p < CAP; ++p) top[p] = 0;  // 0 ranks below every real key
-    for (int j = lane; j < own; j += 32) {
-        uint64_t key = rank_key(block_scores[static_cast<long long>(b) * N + j], j);
-        if (key > top[CAP - 1]) {
-            bool ins = false;
-#pragma unroll
-            for (int p = 0; p < CAP; ++p) {
-                const bool take = ins || key > top[p];
-                if (take) {
-                    const uint64_t t = top[p];
-                    top[p] = key;
-                    key = t;
-                    ins = true;
-                }
-            }
-        }
-    }
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ uint64_t wbest[32];
+    __shared__ int sel[kMaxK + 1];
+    const float *sc = block_scores + static_cast<long long>(b) * N;
     const int m = min(K, own + 1) - 1;
-    __shared__ int sel[kMaxK];
+    // candidates of this thread: j = tid, tid + 1024, ...  (own <= 8192 -> <= 8)
+    uint64_t mine[8];
+    int nm = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const int j = tid + q * kSelThreads;
+        mine[q] = j < own ? rank_key(sc[j], j) : 0;
+        nm += j < own;
+    }
     for (int p = 0; p < m; ++p) {
-        uint64_t best = top[0];
+        uint64_t best = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) best = mine[q] > best ? mine[q] : best;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const uint64_t other = shfl_xor_u64(best, o);
             best = other > best ? other : best;
         }
-        if (top[0] == best && best != 0) {  // keys are unique: exactly one lane pops
+        if (lane == 0) wbest[warp] = best;
+        __syncthreads();
+        if (warp == 0) {
+            uint64_t v = wbest[lane];
 #pragma unroll
-            for (int q = 0; q < CAP - 1; ++q) top[q] = top[q + 1];
-            top[CAP - 1] = 0;
+            for (int o = 16; o > 0; o >>= 1) {
+                const uint64_t other = shfl_xor_u64(v, o);
+                v = other > v ? other : v;
+            }
+            if (lane == 0) wbest[0] = v;
         }
-        if (lane == 0) sel[p] = 0x7FFFFFFF - static_cast<int>(static_cast<uint32_t>(best));
+        __syncthreads();
+        const uint64_t win = wbest[0];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (mine[q] == win) mine[q] = 0;  // keys are unique: one owner
+        if (tid == 0) sel[p] = 0x7FFFFFFF - static_cast<int>(static_cast<uint32_t>(win));
+        __syncthreads();
     }
-    __syncwarp();
-    if (lane == 0) {
+    (void)nm;
+    if (tid == 0) {
         sel[m] = own;
         const int n = m + 1;
         for (int a = 1; a < n; ++a) {  // insertion sort, ascending
@@ -163,11 +181,15 @@ __global__ void __launch_bounds__(32) decode_select_kernel(const float *__restri
 }
 
 // ------------------------------------------------------------------------
-// Split-K decode attention.  One CTA per (b, kv head, slot, split of
-// kDecodeKeys keys).  K/V rows staged in shared memory by 16-byte cp.async
-// (coalesced 2*d-byte rows), G query heads share them; fp32 softmax in the
-// log2 domain.  Writes a normalised fp32 partial and its natural-log lse
-// (-inf when the split has no key).
+// Split-K decode attention.  One CTA of 128 threads per (b, kv head, slot,
+// split of kDecodeKeys keys).  K/V rows are staged in shared memory by
+// 16-byte cp.async (coalesced 2*d-byte rows); the G query heads share them.
+// Scores: thread (key = tid/2, half = tid%2) holds its half K row in
+// registers and reads q (pre-scaled, fp32) as broadcast float4; the two
+// halves are summed by a shuffle.  Softmax in the log2 domain, one warp per
+// head.  PV: thread per output column (and key half when d = 64), p read as
+// float4 over heads.  Writes a normalised fp32 partial and its natural-log
+// lse (-inf when the split has no key).
 // ------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(128) decode_attn_kernel(
@@ -176,26 +198,30 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     float *__restrict__ part_o, float *__restrict__ part_lse, int T, int Hq, int Hkv, int block,
     int K, int S, int N, float scale_log2, int *__restrict__ status) {
     constexpr int KS = kDecodeKeys;
-    constexpr int KSTR = D + 8;  // padded K row (bf16) to spread banks
+    constexpr int KSTR = D + 8;       // padded K row (bf16) to spread banks
+    constexpr int HALF = D / 2;       // elements of a half row
+    constexpr int NH = 128 / D;       // key halves in the PV phase
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int G = Hq / Hkv;
-    float *qs = reinterpret_cast<float *>(smem_raw);                       // [G][D]
-    float *ps = qs + G * D;                                                 // [G][KS]
-    float *ms = ps + G * KS;                                                // [G]
-    float *ls = ms + G;                                                     // [G]
+    const int GP = (G + 3) & ~3;      // heads padded to a float4
+    float *qs = reinterpret_cast<float *>(smem_raw);   // [G][D]
+    float *ps = qs + G * D;                             // [KS][GP]
+    float *ms = ps + KS * GP;                           // [G]
+    float *ls = ms + G;                                 // [G]
+    float *red = ls + G;                                // [NH-1][G][D] (d = 64 only)
     __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(
-        (reinterpret_cast<uintptr_t>(ls + G) + 15) & ~static_cast<uintptr_t>(15));  // [KS][KSTR]
-    __nv_bfloat16 *Vs = Ks + KS * KSTR;                                     // [KS][D]
+        (reinterpret_cast<uintptr_t>(red + (NH - 1) * G * D) + 15) & ~static_cast<uintptr_t>(15));
+    __nv_bfloat16 *Vs = Ks + KS * KSTR;                 // [KS][D]
 
     const int tid = threadIdx.x;
     int idx = blockIdx.x;
-    const int p = idx % S;
+    const int sp = idx % S;
     idx /= S;
     const int s = idx % K;
     idx /= K;
     const int hk = idx % Hkv;
     const int b = idx / Hkv;
-    const long long prow = (static_cast<long long>(b) * K + s) * S + p;  // partial row
+    const long long prow = (static_cast<long long>(b) * K + s) * S + sp;  // partial row
     const int t = T - 1;
     const int j = ids[static_cast<long long>(b) * K + s];
     int nk = 0;
@@ -203,7 +229,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     if (j >= N || j < -1) {
         if (tid == 0) atomicOr(status, kDevBadIds);
     } else if (j >= 0) {
-        k0 = static_cast<long long>(j) * block + static_cast<long long>(p) * KS;
+        k0 = static_cast<long long>(j) * block + static_cast<long long>(sp) * KS;
         long long k1 = k0 + KS;
         const long long blk_end = static_cast<long long>(j + 1) * block;
         if (k1 > blk_end) k1 = blk_end;
@@ -215,7 +241,6 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
         for (int g = tid; g < G; g += blockDim.x) part_lse[prow * Hq + hk * G + g] = -INFINITY;
         return;
     }
-    // stage K and V rows of this split, and the G query rows (pre-scaled)
     constexpr int PIECES = D / 8;  // 16-byte pieces per row
     const __nv_bfloat16 *kbase = k + ((static_cast<long long>(b) * T + k0) * Hkv + hk) * D;
     const __nv_bfloat16 *vbase = v + ((static_cast<long long>(b) * T + k0) * Hkv + hk) * D;
@@ -237,36 +262,60 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
 
-    // scores (log2 domain): ps[g][key]
-    for (int e = tid; e < G * KS; e += blockDim.x) {
-        const int g = e / KS, key = e % KS;
-        float acc = -INFINITY;
-        if (key < nk) {
-            acc = 0.f;
-            const uint4 *kr = reinterpret_cast<const uint4 *>(Ks + key * KSTR);
-            const float *qg = qs + g * D;
-#pragma unroll 4
-            for (int c = 0; c < PIECES; ++c) {
+    // ---- scores: ps[key][g] (log2 domain)
+    {
+        const int key = tid >> 1, half = tid & 1;
+        const bool kv_ok = key < nk;
+        uint4 kr[HALF / 8];
+#pragma unroll
+        for (int c = 0; c < HALF / 8; ++c)
+            kr[c] = kv_ok ? *reinterpret_cast<const uint4 *>(Ks + key * KSTR + half * HALF + c * 8)
+                          : make_uint4(0, 0, 0, 0);
+        for (int g0 = 0; g0 < G; g0 += 8) {
+            float acc[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+#pragma unroll
+            for (int c = 0; c < HALF / 8; ++c) {
                 float kf[8];
                 bf16x8_to_f32(kr[c], kf);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) acc = fmaf(qg[c * 8 + u], kf[u], acc);
+                for (int x = 0; x < 8; ++x) {
+                    if (g0 + x < G) {
+                        const float4 *qp = reinterpret_cast<const float4 *>(qs + (g0 + x) * D + half * HALF + c * 8);
+                        const float4 qa = qp[0], qb = qp[1];
+                        acc[x] = fmaf(qa.x, kf[0], acc[x]);
+                        acc[x] = fmaf(qa.y, kf[1], acc[x]);
+                        acc[x] = fmaf(qa.z, kf[2], acc[x]);
+                        acc[x] = fmaf(qa.w, kf[3], acc[x]);
+                        acc[x] = fmaf(qb.x, kf[4], acc[x]);
+                        acc[x] = fmaf(qb.y, kf[5], acc[x]);
+                        acc[x] = fmaf(qb.z, kf[6], acc[x]);
+                        acc[x] = fmaf(qb.w, kf[7], acc[x]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int x = 0; x < 8; ++x) acc[x] += __shfl_xor_sync(0xFFFFFFFFu, acc[x], 1);
+            if (half == 0) {
+#pragma unroll
+                for (int x = 0; x < 8; ++x)
+                    if (g0 + x < G) ps[key * GP + g0 + x] = kv_ok ? acc[x] : -INFINITY;
             }
         }
-        ps[e] = acc;
     }
     __syncthreads();
-    // per-head max and sum (one warp per head)
+    // ---- per-head max and sum (one warp per head), p in place
     const int warp = tid / 32, lane = tid % 32;
     for (int g = warp; g < G; g += blockDim.x / 32) {
         float mx = -INFINITY;
-        for (int key = lane; key < nk; key += 32) mx = fmaxf(mx, ps[g * KS + key]);
+        for (int key = lane; key < nk; key += 32) mx = fmaxf(mx, ps[key * GP + g]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
         float sum = 0.f;
         for (int key = lane; key < KS; key += 32) {
-            const float pv = key < nk ? exp2f(ps[g * KS + key] - mx) : 0.f;
-            ps[g * KS + key] = pv;
+            const float pv = key < nk ? exp2f(ps[key * GP + g] - mx) : 0.f;
+            ps[key * GP + g] = pv;
             sum += pv;
         }
 #pragma unroll
@@ -277,13 +326,48 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
         }
     }
     __syncthreads();
-    // out[g][c] = sum_key p[g][key] * V[key][c] / l[g]
-    for (int e = tid; e < G * D; e += blockDim.x) {
-        const int g = e / D, c = e % D;
-        float acc = 0.f;
-        const float *pg = ps + g * KS;
-        for (int key = 0; key < nk; ++key) acc = fmaf(pg[key], __bfloat162float(Vs[key * D + c]), acc);
-        part_o[(prow * Hq + hk * G + g) * D + c] = acc / ls[g];
+    // ---- out[g][c] = sum_key p[key][g] * V[key][c] / l[g]
+    {
+        const int c = tid % D, kh = tid / D;  // column, key half (NH halves)
+        const int kb = kh * (KS / NH), ke = min(nk, kb + KS / NH);
+        for (int g0 = 0; g0 < G; g0 += 8) {
+            float acc[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+            for (int key = kb; key < ke; ++key) {
+                const float vv = __bfloat162float(Vs[key * D + c]);
+                const float4 pa = *reinterpret_cast<const float4 *>(ps + key * GP + g0);
+                acc[0] = fmaf(pa.x, vv, acc[0]);
+                acc[1] = fmaf(pa.y, vv, acc[1]);
+                acc[2] = fmaf(pa.z, vv, acc[2]);
+                acc[3] = fmaf(pa.w, vv, acc[3]);
+                if (g0 + 4 < GP) {
+                    const float4 pb = *reinterpret_cast<const float4 *>(ps + key * GP + g0 + 4);
+                    acc[4] = fmaf(pb.x, vv, acc[4]);
+                    acc[5] = fmaf(pb.y, vv, acc[5]);
+                    acc[6] = fmaf(pb.z, vv, acc[6]);
+                    acc[7] = fmaf(pb.w, vv, acc[7]);
+                }
+            }
+            if (NH > 1 && kh > 0) {
+#pragma unroll
+                for (int x = 0; x < 8; ++x)
+                    if (g0 + x < G) red[((kh - 1) * G + g0 + x) * D + c] = acc[x];
+            }
+            if (NH > 1) __syncthreads();
+            if (kh == 0) {
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const int g = g0 + x;
+                    if (g < G) {
+                        float a = acc[x];
+                        for (int h2 = 1; h2 < NH; ++h2) a += red[((h2 - 1) * G + g) * D + c];
+                        part_o[(prow * Hq + hk * G + g) * D + c] = a / ls[g];
+                    }
+                }
+            }
+            if (NH > 1) __syncthreads();
+        }
     }
     for (int g = tid; g < G; g += blockDim.x)
         part_lse[prow * Hq + hk * G + g] = (ms[g] + log2f(ls[g])) * kLn2;
@@ -367,6 +451,82 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
         for (int x = 0; x < VEC; x += 4)
             *reinterpret_cast<float4 *>(dst + x) = make_float4(acc[x], acc[x + 1], acc[x + 2], acc[x + 3]);
     }
+}
+
+// Few query rows (decode): one CTA of 8 warps per (row, head); warp w merges
+// partials p = w, w+8, ... of that head and the warps' sums are added in
+// shared memory.  Same arithmetic as lse_combine_kernel.
+template <typename PT, int D>
+__global__ void __launch_bounds__(256) lse_combine_split_kernel(
+    const PT *__restrict__ part_o, const float *__restrict__ part_lse,
+    const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
+    int K, int S) {
+    constexpr int PER = D / 32;  // elements per lane
+    extern __shared__ float wsm[];                // [P] weights, then [8][D] sums
+    const long long row = blockIdx.x;
+    const int h = blockIdx.y;
+    const int P = K * S;
+    float *acc_s = wsm + ((P + 3) & ~3);
+    __shared__ float L_s;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int pp = tid; pp < P; pp += blockDim.x) {
+        const int si = pp / S;
+        float l = -INFINITY;
+        if (ids[row * K + si] >= 0) l = part_lse[((row * K + si) * S + pp % S) * Hq + h];
+        wsm[pp] = l;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        float mx = -INFINITY;
+        for (int pp = lane; pp < P; pp += 32) mx = fmaxf(mx, wsm[pp]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        float sum = 0.f;
+        for (int pp = lane; pp < P; pp += 32) {
+            const float l = wsm[pp];
+            if (l != -INFINITY) sum += exp2f((l - mx) * kLog2e);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        const float L = mx == -INFINITY ? -INFINITY : mx + log2f(sum) * kLn2;
+        __syncwarp();
+        for (int pp = lane; pp < P; pp += 32) {
+            const float l = wsm[pp];
+            wsm[pp] = (l == -INFINITY) ? 0.f : exp2f((l - L) * kLog2e);
+        }
+        if (lane == 0) L_s = L;
+    }
+    __syncthreads();
+    float acc[PER];
+#pragma unroll
+    for (int x = 0; x < PER; ++x) acc[x] = 0.f;
+    const long long pstride = static_cast<long long>(Hq) * D;
+    const PT *src = part_o + (row * K * S * Hq + h) * static_cast<long long>(D) + lane * PER;
+#pragma unroll 4
+    for (int pp = warp; pp < P; pp += 8) {
+        const float wgt = wsm[pp];
+        const PT *sp = src + pp * pstride;
+        float f[PER];
+        if (sizeof(PT) == 4 && PER == 4) {
+            const float4 u = *reinterpret_cast<const float4 *>(sp);
+            f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+        } else {
+#pragma unroll
+            for (int x = 0; x < PER; ++x) f[x] = static_cast<float>(sp[x]);
+        }
+#pragma unroll
+        for (int x = 0; x < PER; ++x) acc[x] += wgt != 0.f ? wgt * f[x] : 0.f;
+    }
+#pragma unroll
+    for (int x = 0; x < PER; ++x) acc_s[warp * D + lane * PER + x] = acc[x];
+    __syncthreads();
+    for (int c = tid; c < D; c += blockDim.x) {
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) a += acc_s[w * D + c];
+        out[(row * Hq + h) * static_cast<long long>(D) + c] = a;
+    }
+    if (tid == 0) lse_out[row * Hq + h] = L_s;
 }
 
 // ------------------------------------------------------------------------
@@ -568,20 +728,18 @@ __global__ void __launch_bounds__(256) attn_items_kernel(const int *__restrict__
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k_idx,
                                float *block_scores, int num_sms, cudaStream_t st) {
+    (void)num_sms;
     const int own = (sh.T - 1) / sh.block;
     if (own > 0) {
-        const long long work = static_cast<long long>(sh.Bt) * own;
-        long long blocks = (work + 7) / 8;
-        const long long cap = static_cast<long long>(num_sms) * 8;
-        if (blocks > cap) blocks = cap;
+        const long long grid = static_cast<long long>(sh.Bt) * own;
         const auto *qi = static_cast<const __nv_bfloat16 *>(q_idx);
         const auto *ki = static_cast<const __nv_bfloat16 *>(k_idx);
         if (sh.d_idx == 128)
-            decode_index_scan_kernel<128><<<static_cast<int>(blocks), 256, 0, st>>>(
-                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N);
+            decode_index_scan_kernel<128><<<static_cast<unsigned>(grid), 256, 0, st>>>(
+                qi, ki, block_scores, sh.T, sh.block, own, sh.N);
         else
-            decode_index_scan_kernel<64><<<static_cast<int>(blocks), 256, 0, st>>>(
-                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N);
+            decode_index_scan_kernel<64><<<static_cast<unsigned>(grid), 256, 0, st>>>(
+                qi, ki, block_scores, sh.T, sh.block, own, sh.N);
     }
     return cudaGetLastError();
 }
@@ -589,18 +747,16 @@ cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k
 cudaError_t launch_decode_select(const Shape &sh, const float *block_scores, int32_t *ids,
                                  cudaStream_t st) {
     const int own = (sh.T - 1) / sh.block;
-    if (sh.K <= 8)
-        decode_select_kernel<7><<<sh.Bt, 32, 0, st>>>(block_scores, ids, sh.N, own, sh.K);
-    else if (sh.K <= 16)
-        decode_select_kernel<15><<<sh.Bt, 32, 0, st>>>(block_scores, ids, sh.N, own, sh.K);
-    else
-        decode_select_kernel<31><<<sh.Bt, 32, 0, st>>>(block_scores, ids, sh.N, own, sh.K);
+    decode_select_kernel<<<sh.Bt, kSelThreads, 0, st>>>(block_scores, ids, sh.N, own, sh.K);
     return cudaGetLastError();
 }
 
 size_t decode_attn_smem_bytes(const Shape &sh) {
     const int G = sh.G;
-    size_t f = static_cast<size_t>(G) * sh.d + static_cast<size_t>(G) * kDecodeKeys + 2 * G;
+    const int GP = (G + 3) & ~3;
+    const int NH = 128 / sh.d;
+    size_t f = static_cast<size_t>(G) * sh.d + static_cast<size_t>(kDecodeKeys) * GP + 2 * G +
+               static_cast<size_t>(NH - 1) * G * sh.d;
     size_t bytes = align_up(f * 4, 16);
     bytes += static_cast<size_t>(kDecodeKeys) * (sh.d + 8) * 2 + static_cast<size_t>(kDecodeKeys) * sh.d * 2;
     return bytes;
@@ -635,6 +791,25 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            const float *part_lse, const int32_t *ids, float *out, float *lse,
                            int S, cudaStream_t st) {
     const long long rows = static_cast<long long>(sh.Bt) * sh.n_q;
+    if (rows * sh.Hq < 4096 && !part_bf16) {
+        // few rows: split the partials of each (row, head) across 8 warps
+        const int P = sh.K * S;
+        const size_t smem = (static_cast<size_t>((P + 3) & ~3) + 8 * sh.d) * sizeof(float);
+        const dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>(sh.Hq));
+        const auto *po = static_cast<const float *>(part_o);
+        if (sh.d == 128) {
+            cudaFuncSetAttribute(lse_combine_split_kernel<float, 128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            lse_combine_split_kernel<float, 128><<<grid, 256, smem, st>>>(po, part_lse, ids, out,
+                                                                         lse, sh.Hq, sh.K, S);
+        } else {
+            cudaFuncSetAttribute(lse_combine_split_kernel<float, 64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            lse_combine_split_kernel<float, 64><<<grid, 256, smem, st>>>(po, part_lse, ids, out,
+                                                                        lse, sh.Hq, sh.K, S);
+        }
+        return cudaGetLastError();
+    }
     // heads per CTA: all of them when there are many rows, else fewer so the
     // grid still covers the SMs a few times
     int HG = sh.Hq;

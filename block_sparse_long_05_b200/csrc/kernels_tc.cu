@@ -426,11 +426,13 @@ struct AttnParams {
     float scale_log2;
 };
 
-// Per-chunk token table, filled by the gathering warpgroup.
-struct ChunkRows {
-    long long qoff[128];  // element offset of the token's first head of group hk in q
-    int entry[128];       // list entry = partial row (b*n_q + i)*K + slot, or -1
-    int t[128];           // query position, or -1
+// Token table of one work item (at most kItemTokens hit-list entries),
+// built once per item in shared memory.
+constexpr int kItemTokens = 1024;
+struct ItemRows {
+    long long qoff[kItemTokens];  // element offset of the token's head group hk in q
+    int entry[kItemTokens];       // list entry = partial row (b*n_q + i)*K + slot, or -1
+    int t[kItemTokens];           // query position, or -1
 };
 
 template <int D>
@@ -451,8 +453,8 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
     unsigned char *q_s = kv_s + KVST * 2 * kv_tile;               // [wg][buf] Q tiles
     const int QBUF = streamed ? 1 : 2;
     unsigned char *tail = q_s + 2 * QBUF * QBYTES;
-    ChunkRows *rows_s = reinterpret_cast<ChunkRows *>(tail);      // [wg][buf]
-    uint64_t *kvfull = reinterpret_cast<uint64_t *>(rows_s + 2 * QBUF);  // [2]
+    ItemRows *tab = reinterpret_cast<ItemRows *>(tail);
+    uint64_t *kvfull = reinterpret_cast<uint64_t *>(tab + 1);     // [2]
     uint64_t *bar_s = kvfull + 2;                                 // [wg]
     uint64_t *bar_o = kvfull + 4;                                 // [wg]
     int *sh_item = reinterpret_cast<int *>(kvfull + 6);
@@ -513,41 +515,18 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
         ++kv_issue;
     };
 
-    // Token table of chunk `c` into rows_s[wg][buf], then the cp.async gather
-    // of its 128 Q rows into q_s[wg][buf].  Called by one whole warpgroup.
-    auto gather = [&](int buf, int hk, int b, int list_base, int c, int ntok) {
-        ChunkRows &cr = rows_s[wg * QBUF + buf];
-        const int tok0 = c * TOK;
-        if (wtid < TOK) {
-            int e = -1, t = -1;
-            long long qoff = 0;
-            if (tok0 + wtid < ntok) {
-                e = p.entries[list_base + tok0 + wtid];
-                const int qrow = e >= 0 ? e / K : -1;
-                const int bi = qrow >= 0 ? qrow / p.n_q : -1;
-                if (e < 0 || bi != b) {
-                    atomicOr(p.status, kDevBadIds);
-                    e = -1;
-                } else {
-                    t = p.T - p.n_q + (qrow - bi * p.n_q);
-                    qoff = (static_cast<long long>(qrow) * p.Hq + static_cast<long long>(hk) * G) * D;
-                }
-            }
-            cr.entry[wtid] = e;
-            cr.t[wtid] = t;
-            cr.qoff[wtid] = qoff;
-        }
-        named_barrier(wg_bar, 128);
+    // cp.async gather of the 128 Q rows of chunk `c` into q_s[wg][buf]: one
+    // thread per row (token tk = row / G, head g = row % G), 2*D contiguous
+    // bytes each.  Called by one whole warpgroup.
+    auto gather = [&](int buf, int c) {
         unsigned char *dst_base = q_s + (wg * QBUF + buf) * QBYTES;
-#pragma unroll 4
-        for (int pc = wtid; pc < 128 * PPR; pc += 128) {
-            const int r = pc / PPR, cc = pc % PPR;
-            const int tk = r >> p.log2G, gg = r & (G - 1);
-            const bool ok = cr.t[tk] >= 0;
-            const __nv_bfloat16 *src = p.q + (ok ? cr.qoff[tk] + gg * D + cc * 8 : 0);
-            cp_async_16(dst_base + (cc / 8) * kRegionBytes + sw128_offset(r, cc % 8), src,
-                        ok ? 16u : 0u);
-        }
+        const int ti = c * TOK + tok;
+        const bool ok = tab->t[ti] >= 0;
+        const __nv_bfloat16 *src = p.q + (ok ? tab->qoff[ti] + g * D : 0);
+#pragma unroll
+        for (int cc = 0; cc < PPR; ++cc)
+            cp_async_16(dst_base + (cc / 8) * kRegionBytes + sw128_offset(row, cc % 8),
+                        src + (ok ? cc * 8 : 0), ok ? 16u : 0u);
         cp_async_commit();
     };
 
@@ -570,7 +549,29 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
         const int n_steps = streamed ? pairs * p.NS : my_chunks;
 
         if (tid == 0) issue_kv(b, j, hk, 0);
-        if (my_chunks > 0) gather(0, hk, b, list_base, wg, ntok);
+        // token table of the item: coalesced loads of its list entries and
+        // one division per token (tokens past the list end stay invalid)
+        for (int i = tid; i < n_chunks * TOK; i += blockDim.x) {
+            int e = -1, t = -1;
+            long long qoff = 0;
+            if (i < ntok) {
+                e = p.entries[list_base + i];
+                const int qrow = e >= 0 ? e / K : -1;
+                const int bi = qrow >= 0 ? qrow / p.n_q : -1;
+                if (e < 0 || bi != b) {
+                    atomicOr(p.status, kDevBadIds);
+                    e = -1;
+                } else {
+                    t = p.T - p.n_q + (qrow - bi * p.n_q);
+                    qoff = (static_cast<long long>(qrow) * p.Hq + static_cast<long long>(hk) * G) * D;
+                }
+            }
+            tab->entry[i] = e;
+            tab->t[i] = t;
+            tab->qoff[i] = qoff;
+        }
+        __syncthreads();
+        if (my_chunks > 0) gather(0, wg);
 
         float m_run = -INFINITY, l_run = 0.f;
         for (int step = 0; step < n_steps; ++step) {
@@ -581,7 +582,7 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
             const int buf = streamed ? 0 : (ci & 1);
             // ---- Q of this chunk: gathered at item start (first chunk), by the
             // previous step's prefetch, or here (streamed: single Q buffer)
-            if (streamed && kt == 0 && ci > 0 && active) gather(0, hk, b, list_base, c, ntok);
+            if (streamed && kt == 0 && ci > 0 && active) gather(0, c);
             if (kt == 0) cp_async_wait_all();
             fence_proxy_async_smem();
             bool ok = true;
@@ -590,13 +591,14 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                 // lockstep: both warpgroups use this sub-tile; the other stage
                 // is free once both finished their PV of the previous step
                 st = kv_use % KVST;
-                ok = mbar_wait(kvfull + st, (kv_use / KVST) & 1, abort_flag, p.status);
+                if (tid == 0) ok = mbar_wait(kvfull + st, (kv_use / KVST) & 1, abort_flag, p.status);
                 ++kv_use;
                 if (__syncthreads_or(!ok)) { aborted = true; break; }
                 if (tid == 0 && step + 1 < n_steps) issue_kv(b, j, hk, (step + 1) % p.NS);
             } else {
-                // one K/V load per item (stage 0), the item_n-th of this CTA
-                if (step == 0) ok = mbar_wait(kvfull, item_n & 1, abort_flag, p.status);
+                // one K/V load per item (stage 0), the item_n-th of this CTA;
+                // one thread polls, the warpgroup barrier releases the rest
+                if (step == 0 && wtid == 0) ok = mbar_wait(kvfull, item_n & 1, abort_flag, p.status);
                 if (named_barrier_or(wg_bar, 128, !ok || *abort_flag)) { aborted = true; break; }
             }
             unsigned char *kd = kv_s + st * 2 * kv_tile;
@@ -613,9 +615,9 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                 umma_commit(bar_s + wg);
             }
             // prefetch the next chunk's Q while this one computes
-            if (!streamed && ci + 1 < my_chunks) gather(buf ^ 1, hk, b, list_base, c + 2, ntok);
+            if (!streamed && ci + 1 < my_chunks) gather(buf ^ 1, c + 2);
             if (active) {
-                ok = mbar_wait(bar_s + wg, s_n & 1, abort_flag, p.status);
+                if (wtid == 0) ok = mbar_wait(bar_s + wg, s_n & 1, abort_flag, p.status);
                 ++s_n;
             }
             if (streamed) {
@@ -625,8 +627,7 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
             }
             if (active) {
                 tc_fence_after();
-                const ChunkRows &cr = rows_s[wg * QBUF + buf];
-                const int t = cr.t[tok];
+                const int t = tab->t[c * TOK + tok];
                 const int lim = t - (j * p.block + kt * NK);  // valid key columns: <= lim
                 // ---- softmax of this row (registers)
                 float sv[128];
@@ -645,11 +646,18 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                     for (int x = 0; x < 128; ++x)
                         if (x > lim) sv[x] = -INFINITY;
                 }
-                float mt = -INFINITY;
+                // row max: four independent chains of 3-input max
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int x = 0; x < 128; ++x)
-                    if (x < NK) mt = fmaxf(mt, sv[x]);
-                mt *= p.scale_log2;
+                for (int x = 0; x < 128; x += 8) {
+                    if (x < NK) {
+                        m4[0] = fmax3(m4[0], sv[x], sv[x + 1]);
+                        m4[1] = fmax3(m4[1], sv[x + 2], sv[x + 3]);
+                        m4[2] = fmax3(m4[2], sv[x + 4], sv[x + 5]);
+                        m4[3] = fmax3(m4[3], sv[x + 6], sv[x + 7]);
+                    }
+                }
+                float mt = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * p.scale_log2;
                 if (kt == 0) {
                     m_run = mt;
                     l_run = 0.f;
@@ -676,22 +684,31 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                     }
                 }
                 const float mref = m_run == -INFINITY ? 0.f : m_run;
-                float lsum = 0.f;
+                const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+                const uint64_t nm2 = f2_pack(-mref, -mref);
+                uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
 #pragma unroll
                 for (int g32 = 0; g32 < 4; ++g32) {  // 32 keys -> 16 packed columns
                     if (g32 * 32 < NK) {
                         uint32_t w16[16];
 #pragma unroll
                         for (int x = 0; x < 16; ++x) {
-                            const float p0 = ex2_approx(fmaf(sv[g32 * 32 + 2 * x], p.scale_log2, -mref));
-                            const float p1 = ex2_approx(fmaf(sv[g32 * 32 + 2 * x + 1], p.scale_log2, -mref));
-                            lsum += p0 + p1;
+                            float a0, a1;
+                            f2_unpack(f2_fma(f2_pack(sv[g32 * 32 + 2 * x], sv[g32 * 32 + 2 * x + 1]), sc2, nm2), a0, a1);
+                            const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+                            if (x & 1)
+                                ls2b = f2_add(ls2b, f2_pack(p0, p1));
+                            else
+                                ls2a = f2_add(ls2a, f2_pack(p0, p1));
                             w16[x] = pack_bf16x2(p0, p1);
                         }
                         tmem_st16(tmem_s + lane_addr + g32 * 16, w16);
                     }
                 }
-                l_run += lsum;
+                float la0, la1, lb0, lb1;
+                f2_unpack(ls2a, la0, la1);
+                f2_unpack(ls2b, lb0, lb1);
+                l_run += (la0 + la1) + (lb0 + lb1);
                 tmem_wait_st();
                 tc_fence_before();
             }
@@ -706,7 +723,7 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                 umma_commit(bar_o + wg);
             }
             if (active) {
-                ok = mbar_wait(bar_o + wg, o_n & 1, abort_flag, p.status);
+                if (wtid == 0) ok = mbar_wait(bar_o + wg, o_n & 1, abort_flag, p.status);
                 ++o_n;
             }
             if (streamed) {
@@ -717,8 +734,7 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
             if (active && kt == p.NS - 1) {
                 tc_fence_after();
                 // ---- epilogue: normalised bf16 partial and its lse
-                const ChunkRows &cr = rows_s[wg * QBUF + buf];
-                const int e = cr.entry[tok];
+                const int e = tab->entry[c * TOK + tok];
                 const bool valid = e >= 0;
                 const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
                 const long long prow = static_cast<long long>(valid ? e : 0) * p.Hq +
@@ -730,15 +746,18 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                     tmem_ld32(tmem_o + lane_addr + cc * 32, v);
                     tmem_wait_ld();
                     if (valid) {
+                        const uint64_t il2 = f2_pack(inv_l, inv_l);
+                        uint32_t w[16];
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint4 u;
-                            u.x = pack_bf16x2(__uint_as_float(v[q4 * 8 + 0]) * inv_l, __uint_as_float(v[q4 * 8 + 1]) * inv_l);
-                            u.y = pack_bf16x2(__uint_as_float(v[q4 * 8 + 2]) * inv_l, __uint_as_float(v[q4 * 8 + 3]) * inv_l);
-                            u.z = pack_bf16x2(__uint_as_float(v[q4 * 8 + 4]) * inv_l, __uint_as_float(v[q4 * 8 + 5]) * inv_l);
-                            u.w = pack_bf16x2(__uint_as_float(v[q4 * 8 + 6]) * inv_l, __uint_as_float(v[q4 * 8 + 7]) * inv_l);
-                            *reinterpret_cast<uint4 *>(dst + cc * 32 + q4 * 8) = u;
+                        for (int x = 0; x < 16; ++x) {
+                            float a0, a1;
+                            f2_unpack(f2_mul(f2_pack(__uint_as_float(v[2 * x]), __uint_as_float(v[2 * x + 1])), il2), a0, a1);
+                            w[x] = pack_bf16x2(a0, a1);
                         }
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            *reinterpret_cast<uint4 *>(dst + cc * 32 + q4 * 8) =
+                                make_uint4(w[q4 * 4], w[q4 * 4 + 1], w[q4 * 4 + 2], w[q4 * 4 + 3]);
                     }
                 }
                 if (valid)
@@ -827,7 +846,12 @@ size_t prefill_attn_smem_bytes(const Shape &sh) {
     const int QBUF = NS > 1 ? 1 : 2;
     const size_t kv_tile = static_cast<size_t>(NK) * 128 * (sh.d / 64);
     const size_t q = static_cast<size_t>(sh.d / 64) * kRegionBytes;
-    return 1024 + KVST * 2 * kv_tile + 2 * QBUF * q + 2 * QBUF * sizeof(ChunkRows) + 64 + 32;
+    return 1024 + KVST * 2 * kv_tile + 2 * QBUF * q + sizeof(ItemRows) + 64 + 32;
+}
+
+int prefill_attn_rows_per_item(int G) {
+    const int tok = 128 / G;
+    return 16 * tok < kItemTokens ? 16 * tok : kItemTokens;
 }
 
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,

@@ -29,7 +29,7 @@ msa_status validate(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_idx, i
     const long long N = (static_cast<long long>(T) + block - 1) / block;
     if (static_cast<long long>(Bt) * T >= (1ll << 31)) return MSA_ERR_UNSUPPORTED;
     if (static_cast<long long>(Bt) * n_q * K >= (1ll << 31)) return MSA_ERR_UNSUPPORTED;
-    if (n_q > 1 && N > kMaxBlocksPrefill) return MSA_ERR_UNSUPPORTED;
+    if (N > kMaxBlocksPrefill) return MSA_ERR_UNSUPPORTED;
     int G = 1;
     if (need_attn) {
         G = Hq / Hkv;
@@ -59,7 +59,7 @@ WsLayout layout_for(const Shape &sh, bool with_attn) {
     };
     const long long pairs = static_cast<long long>(sh.Bt) * sh.N;
     L.n_chunks = (sh.n_q + kInvRows - 1) / kInvRows;
-    L.rows_per_item = with_attn ? 16 * (128 / sh.G) : 128;  // 16 chunks of 128 rows
+    L.rows_per_item = with_attn ? prefill_attn_rows_per_item(sh.G) : 128;
     L.max_items = static_cast<int>((static_cast<long long>(sh.Bt) * sh.n_q * sh.K + L.rows_per_item - 1) /
                                        L.rows_per_item +
                                    pairs);

@@ -12,7 +12,7 @@ constexpr int kDevTimeout = 1;
 constexpr int kDevBadIds = 2;
 
 constexpr int kMaxK = 32;          // top-K capacity of the register lists
-constexpr int kMaxBlocksPrefill = 8192;  // N limit of the inversion's shared histograms
+constexpr int kMaxBlocksPrefill = 8192;  // N limit (inversion histograms, decode select)
 constexpr int kInvRows = 128;      // query rows per inversion chunk (4 warps x 32)
 constexpr int kDecodeKeys = 64;    // keys per split of the decode attention kernel
 

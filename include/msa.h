@@ -17,8 +17,9 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *    never allocates, frees or retains memory; it keeps no global mutable
- *    state, so calls on different workspaces may run concurrently.
+ *    never allocates, frees or retains memory and (apart from the
+ *    no-allocation decode entry point below) keeps no global mutable state,
+ *    so calls on different workspaces may run concurrently.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
  *    asynchronous on that stream and returns after enqueueing its kernels.
  *  - Layouts are row-major and contiguous, bf16 means IEEE bfloat16 bits:
@@ -39,8 +40,8 @@
  *    q.k_i / sqrt(d) over the keys i <= t of the blocks in ids, output the
  *    weighted sum of v_i (fp32) and lse = ln sum_i exp(q.k_i / sqrt(d)).
  *  - Supported shapes: d, d_idx in {64, 128}; block in {32, 64} or a
- *    multiple of 128; 1 <= K <= 32; 128 % (Hq/Hkv) == 0; N <= 8192 for
- *    prefill (n_q > 1); Bt*T < 2^31 and Bt*n_q*K < 2^31.  Anything else
+ *    multiple of 128; 1 <= K <= 32; 128 % (Hq/Hkv) == 0; N <= 8192;
+ *    Bt*T < 2^31 and Bt*n_q*K < 2^31.  Anything else
  *    returns MSA_ERR_UNSUPPORTED before any work is enqueued.  Tensor base
  *    pointers must be 16-byte aligned (MSA_ERR_INVALID_ARG otherwise).
  *  - Errors found on the host return immediately (nothing enqueued).  Errors a
