@@ -446,12 +446,12 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
     const uint32_t kv_tile = static_cast<uint32_t>(NK) * 128u * DREG;  // one of K or V
     const bool streamed = p.NS > 1;
     const int KVST = streamed ? 2 : 1;
+    const int QBUF = streamed ? 1 : 2;
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = align1024(smem_raw);
     unsigned char *kv_s = base;                                   // KVST x (K tile, V tile)
     unsigned char *q_s = kv_s + KVST * 2 * kv_tile;               // [wg][buf] Q tiles
-    const int QBUF = streamed ? 1 : 2;
     unsigned char *tail = q_s + 2 * QBUF * QBYTES;
     ItemRows *tab = reinterpret_cast<ItemRows *>(tail);
     uint64_t *kvfull = reinterpret_cast<uint64_t *>(tab + 1);     // [2]
@@ -499,6 +499,7 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
     uint32_t kv_issue = 0, kv_use = 0, s_n = 0, o_n = 0, item_n = 0;
     int armed_parity[2] = {-1, -1};
     bool aborted = false;
+    int cur_b = 0, cur_j = 0, cur_hk = 0;
 
     // K/V loads of sub-tile kt of block (b, j), kv head hk (thread 0 only).
     auto issue_kv = [&](int b, int j, int hk, int kt) {
@@ -515,19 +516,259 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
         ++kv_issue;
     };
 
-    // cp.async gather of the 128 Q rows of chunk `c` into q_s[wg][buf]: one
-    // thread per row (token tk = row / G, head g = row % G), 2*D contiguous
-    // bytes each.  Called by one whole warpgroup.
+    // cp.async gather of the 128 Q rows of chunk `c` (row = tk*G + g) into
+    // q_s[wg][buf].  Piece pc = wtid + 128*k is 16-byte chunk pc % PPR of row
+    // pc / PPR, so one warp instruction covers whole 2*D-byte rows (coalesced).
+    // Called by one whole warpgroup.
     auto gather = [&](int buf, int c) {
         unsigned char *dst_base = q_s + (wg * QBUF + buf) * QBYTES;
-        const int ti = c * TOK + tok;
-        const bool ok = tab->t[ti] >= 0;
-        const __nv_bfloat16 *src = p.q + (ok ? tab->qoff[ti] + g * D : 0);
-#pragma unroll
-        for (int cc = 0; cc < PPR; ++cc)
-            cp_async_16(dst_base + (cc / 8) * kRegionBytes + sw128_offset(row, cc % 8),
-                        src + (ok ? cc * 8 : 0), ok ? 16u : 0u);
+#pragma unroll 4
+        for (int pc = wtid; pc < 128 * PPR; pc += 128) {
+            const int r = pc / PPR, cc = pc % PPR;
+            const int ti = c * TOK + (r >> p.log2G);
+            const bool ok = tab->t[ti] >= 0;
+            const __nv_bfloat16 *src = p.q + (ok ? tab->qoff[ti] + (r & (G - 1)) * D + cc * 8 : 0);
+            cp_async_16_ca(dst_base + (cc / 8) * kRegionBytes + sw128_offset(r, cc % 8), src,
+                           ok ? 16u : 0u);
+        }
         cp_async_commit();
+    };
+
+    // S = Q K^T for this warpgroup (its leader thread issues).
+    auto issue_s = [&](int buf, const unsigned char *kd) {
+        if (wtid == 0) {
+            tc_fence_after();
+            const uint32_t qa = smem_addr(q_s + (wg * QBUF + buf) * QBYTES), ka = smem_addr(kd);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                umma_bf16(tmem_s, sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
+                          sdesc_sw128(ka + (kk / 4) * NK * 128 + (kk % 4) * 32, 16, 1024), idesc_s,
+                          kk > 0 ? 1u : 0u);
+            umma_commit(bar_s + wg);
+        }
+    };
+
+    // O (+)= P V, P read from tensor memory (over S).
+    auto issue_pv = [&](const unsigned char *vd, bool first) {
+        if (wtid == 0) {
+            tc_fence_after();
+            const uint32_t va = smem_addr(vd);
+            for (int kk = 0; kk < NK / 16; ++kk)
+                umma_bf16_tmem_a(tmem_o, tmem_s + kk * 8,
+                                 sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
+                                 idesc_o, (!first || kk > 0) ? 1u : 0u);
+            umma_commit(bar_o + wg);
+        }
+    };
+
+    // Warpgroup-wide bounded wait on one of its mbarriers (one thread polls).
+    auto wait_wg = [&](uint64_t *bar, uint32_t parity) -> bool {
+        bool ok = true;
+        if (wtid == 0) ok = mbar_wait(bar, parity, abort_flag, p.status);
+        return !named_barrier_or(wg_bar, 128, !ok || *abort_flag);
+    };
+
+    // Softmax of this thread's row of S (sub-tile kt of chunk c): P over S in
+    // tensor memory as bf16, running max m_run / sum l_run (log2 domain).
+    auto softmax = [&](int c, int kt, float &m_run, float &l_run) {
+        tc_fence_after();
+        const int t = tab->t[c * TOK + tok];
+        const int lim = t - (cur_j * p.block + kt * NK);  // valid key columns: <= lim
+        const bool masked = lim < NK - 1;
+        // pass 1 over S (32 columns at a time): row max
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        for (int cc = 0; cc < NK / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tmem_s + lane_addr + cc * 32, v);
+            tmem_wait_ld();
+            float sv[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+                sv[x] = (masked && cc * 32 + x > lim) ? -INFINITY : __uint_as_float(v[x]);
+#pragma unroll
+            for (int x = 0; x < 32; x += 8) {
+                m4[0] = fmax3(m4[0], sv[x], sv[x + 1]);
+                m4[1] = fmax3(m4[1], sv[x + 2], sv[x + 3]);
+                m4[2] = fmax3(m4[2], sv[x + 4], sv[x + 5]);
+                m4[3] = fmax3(m4[3], sv[x + 6], sv[x + 7]);
+            }
+        }
+        const float mt = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * p.scale_log2;
+        if (kt == 0) {
+            m_run = mt;
+            l_run = 0.f;
+        } else {
+            // online softmax across sub-tiles: rescale O only when the max
+            // grew by more than 2^8 (keeps P <= 256; exact up to rounding)
+            float alpha = 1.f;
+            bool need = false;
+            if (mt > m_run + 8.f) {
+                alpha = ex2_approx(m_run - mt);
+                m_run = mt;
+                l_run *= alpha;
+                need = true;
+            }
+            if (__any_sync(0xFFFFFFFFu, need)) {
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem_o + lane_addr + cc * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
+                    tmem_st32(tmem_o + lane_addr + cc * 32, v);
+                }
+                tmem_wait_st();
+            }
+        }
+        const float mref = m_run == -INFINITY ? 0.f : m_run;
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(-mref, -mref);
+        uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
+        // pass 2 over S: P = 2^(s*c - m) as bf16, written over the columns of
+        // S already consumed (32 keys -> 16 packed columns)
+        for (int cc = 0; cc < NK / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tmem_s + lane_addr + cc * 32, v);
+            tmem_wait_ld();
+            uint32_t w16[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                const float s0 = (masked && cc * 32 + 2 * x > lim) ? -INFINITY : __uint_as_float(v[2 * x]);
+                const float s1 = (masked && cc * 32 + 2 * x + 1 > lim) ? -INFINITY : __uint_as_float(v[2 * x + 1]);
+                float a0, a1;
+                f2_unpack(f2_fma(f2_pack(s0, s1), sc2, nm2), a0, a1);
+                const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+                if (x & 1)
+                    ls2b = f2_add(ls2b, f2_pack(p0, p1));
+                else
+                    ls2a = f2_add(ls2a, f2_pack(p0, p1));
+                w16[x] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tmem_s + lane_addr + cc * 16, w16);
+        }
+        float la0, la1, lb0, lb1;
+        f2_unpack(ls2a, la0, la1);
+        f2_unpack(ls2b, lb0, lb1);
+        l_run += (la0 + la1) + (lb0 + lb1);
+        tmem_wait_st();
+        tc_fence_before();
+    };
+
+    // Softmax of a whole block held in one tile (block <= 128): single pass
+    // from registers, no running max.  P over S in tensor memory as bf16.
+    auto softmax_tile = [&](int c, float &m_run, float &l_run) {
+        tc_fence_after();
+        const int t = tab->t[c * TOK + tok];
+        const int lim = t - cur_j * p.block;  // valid key columns: <= lim
+        float sv[128];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            if (cc * 32 < NK) {
+                uint32_t v[32];
+                tmem_ld32(tmem_s + lane_addr + cc * 32, v);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) sv[cc * 32 + x] = __uint_as_float(v[x]);
+            }
+        }
+        tmem_wait_ld();
+        if (lim < NK - 1) {
+#pragma unroll
+            for (int x = 0; x < 128; ++x)
+                if (x > lim) sv[x] = -INFINITY;
+        }
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int x = 0; x < 128; x += 8) {
+            if (x < NK) {
+                m4[0] = fmax3(m4[0], sv[x], sv[x + 1]);
+                m4[1] = fmax3(m4[1], sv[x + 2], sv[x + 3]);
+                m4[2] = fmax3(m4[2], sv[x + 4], sv[x + 5]);
+                m4[3] = fmax3(m4[3], sv[x + 6], sv[x + 7]);
+            }
+        }
+        m_run = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * p.scale_log2;
+        const float mref = m_run == -INFINITY ? 0.f : m_run;
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(-mref, -mref);
+        uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
+#pragma unroll
+        for (int g32 = 0; g32 < 4; ++g32) {  // 32 keys -> 16 packed columns
+            if (g32 * 32 < NK) {
+                uint32_t w16[16];
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    float a0, a1;
+                    f2_unpack(f2_fma(f2_pack(sv[g32 * 32 + 2 * x], sv[g32 * 32 + 2 * x + 1]), sc2, nm2), a0, a1);
+                    const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+                    if (x & 1)
+                        ls2b = f2_add(ls2b, f2_pack(p0, p1));
+                    else
+                        ls2a = f2_add(ls2a, f2_pack(p0, p1));
+                    w16[x] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(tmem_s + lane_addr + g32 * 16, w16);
+            }
+        }
+        float la0, la1, lb0, lb1;
+        f2_unpack(ls2a, la0, la1);
+        f2_unpack(ls2b, lb0, lb1);
+        l_run = (la0 + la1) + (lb0 + lb1);
+        tmem_wait_st();
+        tc_fence_before();
+    };
+
+    // Normalised bf16 partial and its natural-log lse for chunk c.  Each
+    // thread packs its row and writes it to `stage` (the chunk's Q buffer,
+    // dead once S is done) with 16-byte pieces XOR-swizzled by the row; the
+    // warpgroup then reads the tile back two rows per warp instruction and
+    // stores whole rows (the G rows of a token are contiguous in the
+    // partials), so every global store instruction writes 512 contiguous
+    // bytes.
+    auto epilogue = [&](int c, float m_run, float l_run, unsigned char *stage) {
+        tc_fence_after();
+        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        const uint64_t il2 = f2_pack(inv_l, inv_l);
+        unsigned char *srow = stage + row * (D * 2);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tmem_o + lane_addr + cc * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t w[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    float a0, a1;
+                    f2_unpack(f2_mul(f2_pack(__uint_as_float(v[q4 * 8 + 2 * x]), __uint_as_float(v[q4 * 8 + 2 * x + 1])), il2), a0, a1);
+                    w[x] = pack_bf16x2(a0, a1);
+                }
+                const int piece = cc * 4 + q4;
+                *reinterpret_cast<uint4 *>(srow + ((piece ^ (row & (PPR - 1))) << 4)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        const int e = tab->entry[c * TOK + tok];
+        if (e >= 0) {
+            const long long prow = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G + g;
+            p.part_lse[prow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
+        }
+        tc_fence_before();
+        named_barrier(wg_bar, 128);
+        // coalesced copy-out: lane -> (row r = base + lane / PPR, piece lane % PPR)
+        constexpr int RPI = 32 / PPR;  // rows per warp instruction
+        const int wl = wtid & 31, wq = wtid >> 5;
+        const int piece = wl % PPR;
+#pragma unroll 4
+        for (int it = 0; it < 32 / RPI; ++it) {
+            const int r = wq * 32 + it * RPI + wl / PPR;
+            const int er = tab->entry[c * TOK + (r >> p.log2G)];
+            const uint4 u = *reinterpret_cast<const uint4 *>(stage + r * (D * 2) + ((piece ^ (r & (PPR - 1))) << 4));
+            if (er >= 0) {
+                const long long prow = static_cast<long long>(er) * p.Hq + static_cast<long long>(cur_hk) * G + (r & (G - 1));
+                *reinterpret_cast<uint4 *>(p.part_o + prow * D + piece * 8) = u;
+            }
+        }
     };
 
     while (true) {
@@ -538,15 +779,14 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
         const int hk = w / n_items;
         const AttnItem item = p.items[w - hk * n_items];
         const int b = item.pair / p.N, j = item.pair - b * p.N;
+        cur_b = b;
+        cur_j = j;
+        cur_hk = hk;
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
         // chunks of this warpgroup: c = wg, wg + 2, ...
         const int my_chunks = n_chunks > wg ? (n_chunks - wg + 1) / 2 : 0;
-        // steps: with streamed K/V both warpgroups walk (chunk pair, sub-tile)
-        // in lockstep, otherwise each walks its own chunks
-        const int pairs = (n_chunks + 1) / 2;
-        const int n_steps = streamed ? pairs * p.NS : my_chunks;
 
         if (tid == 0) issue_kv(b, j, hk, 0);
         // token table of the item: coalesced loads of its list entries and
@@ -571,204 +811,81 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
             tab->qoff[i] = qoff;
         }
         __syncthreads();
-        if (my_chunks > 0) gather(0, wg);
 
-        float m_run = -INFINITY, l_run = 0.f;
-        for (int step = 0; step < n_steps; ++step) {
-            const int ci = streamed ? step / p.NS : step;   // index among my chunks
-            const int kt = streamed ? step % p.NS : 0;
-            const int c = wg + 2 * ci;                      // chunk index in the item
-            const bool active = c < n_chunks;
-            const int buf = streamed ? 0 : (ci & 1);
-            // ---- Q of this chunk: gathered at item start (first chunk), by the
-            // previous step's prefetch, or here (streamed: single Q buffer)
-            if (streamed && kt == 0 && ci > 0 && active) gather(0, c);
-            if (kt == 0) cp_async_wait_all();
-            fence_proxy_async_smem();
-            bool ok = true;
-            uint32_t st = 0;
-            if (streamed) {
-                // lockstep: both warpgroups use this sub-tile; the other stage
-                // is free once both finished their PV of the previous step
-                st = kv_use % KVST;
+        if (!streamed) {
+            // ---- K/V resident for the whole item; each warpgroup pipelines its
+            // chunks: S(c+1) is issued before the epilogue of c.
+            const unsigned char *kd = kv_s, *vd = kv_s + kv_tile;
+            const int n = my_chunks;
+            if (n > 0) gather(0, wg);
+            for (int ci = 0; ci < n; ++ci) {
+                const int c = wg + 2 * ci, buf = ci & 1;
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                if (ci == 0) {
+                    if (!wait_wg(kvfull, item_n & 1)) { aborted = true; break; }
+                } else {
+                    named_barrier(wg_bar, 128);
+                }
+                issue_s(buf, kd);
+                // next chunk's Q into the other buffer (its S finished a chunk ago)
+                if (ci + 1 < n) gather(buf ^ 1, c + 2);
+                if (!wait_wg(bar_s + wg, s_n & 1)) { aborted = true; break; }
+                ++s_n;
+                float m_run, l_run;
+                softmax_tile(c, m_run, l_run);
+                named_barrier(wg_bar, 128);
+                issue_pv(vd, true);
+                if (!wait_wg(bar_o + wg, o_n & 1)) { aborted = true; break; }
+                ++o_n;
+                epilogue(c, m_run, l_run, q_s + (wg * QBUF + buf) * QBYTES);
+            }
+        } else {
+            // ---- K/V streamed in sub-tiles (double-buffered); both warpgroups
+            // walk (chunk pair, sub-tile) in lockstep with an online softmax.
+            const int pairs = (n_chunks + 1) / 2;
+            const int n_steps = pairs * p.NS;
+            float m_run = -INFINITY, l_run = 0.f;
+            if (my_chunks > 0) gather(0, wg);
+            for (int step = 0; step < n_steps; ++step) {
+                const int ci = step / p.NS, kt = step % p.NS;
+                const int c = wg + 2 * ci;
+                const bool active = c < n_chunks;
+                if (kt == 0 && active && ci > 0) {
+                    named_barrier(wg_bar, 128);  // staged partial of the previous chunk read out
+                    gather(0, c);
+                }
+                if (kt == 0) cp_async_wait_all();
+                fence_proxy_async_smem();
+                const uint32_t st = kv_use % KVST;
+                bool ok = true;
                 if (tid == 0) ok = mbar_wait(kvfull + st, (kv_use / KVST) & 1, abort_flag, p.status);
                 ++kv_use;
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
+                if (__syncthreads_or(!ok || *abort_flag)) { aborted = true; break; }
                 if (tid == 0 && step + 1 < n_steps) issue_kv(b, j, hk, (step + 1) % p.NS);
-            } else {
-                // one K/V load per item (stage 0), the item_n-th of this CTA;
-                // one thread polls, the warpgroup barrier releases the rest
-                if (step == 0 && wtid == 0) ok = mbar_wait(kvfull, item_n & 1, abort_flag, p.status);
-                if (named_barrier_or(wg_bar, 128, !ok || *abort_flag)) { aborted = true; break; }
-            }
-            unsigned char *kd = kv_s + st * 2 * kv_tile;
-            unsigned char *vd = kd + kv_tile;
-            if (active && wtid == 0) {
-                tc_fence_after();
-                const uint32_t qa = smem_addr(q_s + (wg * QBUF + buf) * QBYTES), ka = smem_addr(kd);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_bf16(tmem_s,
-                              sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
-                              sdesc_sw128(ka + (kk / 4) * NK * 128 + (kk % 4) * 32, 16, 1024),
-                              idesc_s, kk > 0 ? 1u : 0u);
-                umma_commit(bar_s + wg);
-            }
-            // prefetch the next chunk's Q while this one computes
-            if (!streamed && ci + 1 < my_chunks) gather(buf ^ 1, c + 2);
-            if (active) {
-                if (wtid == 0) ok = mbar_wait(bar_s + wg, s_n & 1, abort_flag, p.status);
-                ++s_n;
-            }
-            if (streamed) {
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
-            } else {
-                if (named_barrier_or(wg_bar, 128, !ok || *abort_flag)) { aborted = true; break; }
-            }
-            if (active) {
-                tc_fence_after();
-                const int t = tab->t[c * TOK + tok];
-                const int lim = t - (j * p.block + kt * NK);  // valid key columns: <= lim
-                // ---- softmax of this row (registers)
-                float sv[128];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    if (cc * 32 < NK) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem_s + lane_addr + cc * 32, v);
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) sv[cc * 32 + x] = __uint_as_float(v[x]);
-                    }
-                }
-                tmem_wait_ld();
-                if (lim < NK - 1) {
-#pragma unroll
-                    for (int x = 0; x < 128; ++x)
-                        if (x > lim) sv[x] = -INFINITY;
-                }
-                // row max: four independent chains of 3-input max
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int x = 0; x < 128; x += 8) {
-                    if (x < NK) {
-                        m4[0] = fmax3(m4[0], sv[x], sv[x + 1]);
-                        m4[1] = fmax3(m4[1], sv[x + 2], sv[x + 3]);
-                        m4[2] = fmax3(m4[2], sv[x + 4], sv[x + 5]);
-                        m4[3] = fmax3(m4[3], sv[x + 6], sv[x + 7]);
-                    }
-                }
-                float mt = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * p.scale_log2;
-                if (kt == 0) {
-                    m_run = mt;
+                const unsigned char *kd = kv_s + st * 2 * kv_tile;
+                const unsigned char *vd = kd + kv_tile;
+                if (active) issue_s(0, kd);
+                ok = true;
+                if (active && wtid == 0) ok = mbar_wait(bar_s + wg, s_n & 1, abort_flag, p.status);
+                if (active) ++s_n;
+                if (__syncthreads_or(!ok || *abort_flag)) { aborted = true; break; }
+                if (active) softmax(c, kt, m_run, l_run);
+                named_barrier(wg_bar, 128);
+                if (active) issue_pv(vd, kt == 0);
+                ok = true;
+                if (active && wtid == 0) ok = mbar_wait(bar_o + wg, o_n & 1, abort_flag, p.status);
+                if (active) ++o_n;
+                if (__syncthreads_or(!ok || *abort_flag)) { aborted = true; break; }
+                if (active && kt == p.NS - 1) {
+                    epilogue(c, m_run, l_run, q_s + wg * QBUF * QBYTES);
+                    m_run = -INFINITY;
                     l_run = 0.f;
-                } else {
-                    float alpha = 1.f;
-                    bool need = false;
-                    if (mt > m_run + 8.f) {
-                        alpha = ex2_approx(m_run - mt);
-                        m_run = mt;
-                        l_run *= alpha;
-                        need = true;
-                    }
-                    if (__any_sync(0xFFFFFFFFu, need)) {
-                        for (int cc = 0; cc < D / 32; ++cc) {
-                            uint32_t v[32];
-                            tmem_ld32(tmem_o + lane_addr + cc * 32, v);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int x = 0; x < 32; ++x)
-                                v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
-                            tmem_st32(tmem_o + lane_addr + cc * 32, v);
-                        }
-                        tmem_wait_st();
-                    }
                 }
-                const float mref = m_run == -INFINITY ? 0.f : m_run;
-                const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-                const uint64_t nm2 = f2_pack(-mref, -mref);
-                uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
-#pragma unroll
-                for (int g32 = 0; g32 < 4; ++g32) {  // 32 keys -> 16 packed columns
-                    if (g32 * 32 < NK) {
-                        uint32_t w16[16];
-#pragma unroll
-                        for (int x = 0; x < 16; ++x) {
-                            float a0, a1;
-                            f2_unpack(f2_fma(f2_pack(sv[g32 * 32 + 2 * x], sv[g32 * 32 + 2 * x + 1]), sc2, nm2), a0, a1);
-                            const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
-                            if (x & 1)
-                                ls2b = f2_add(ls2b, f2_pack(p0, p1));
-                            else
-                                ls2a = f2_add(ls2a, f2_pack(p0, p1));
-                            w16[x] = pack_bf16x2(p0, p1);
-                        }
-                        tmem_st16(tmem_s + lane_addr + g32 * 16, w16);
-                    }
-                }
-                float la0, la1, lb0, lb1;
-                f2_unpack(ls2a, la0, la1);
-                f2_unpack(ls2b, lb0, lb1);
-                l_run += (la0 + la1) + (lb0 + lb1);
-                tmem_wait_st();
-                tc_fence_before();
-            }
-            named_barrier(wg_bar, 128);
-            if (active && wtid == 0) {
-                tc_fence_after();
-                const uint32_t va = smem_addr(vd);
-                for (int kk = 0; kk < NK / 16; ++kk)
-                    umma_bf16_tmem_a(tmem_o, tmem_s + kk * 8,
-                                     sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
-                                     idesc_o, (kt > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(bar_o + wg);
-            }
-            if (active) {
-                if (wtid == 0) ok = mbar_wait(bar_o + wg, o_n & 1, abort_flag, p.status);
-                ++o_n;
-            }
-            if (streamed) {
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
-            } else {
-                if (named_barrier_or(wg_bar, 128, !ok || *abort_flag)) { aborted = true; break; }
-            }
-            if (active && kt == p.NS - 1) {
-                tc_fence_after();
-                // ---- epilogue: normalised bf16 partial and its lse
-                const int e = tab->entry[c * TOK + tok];
-                const bool valid = e >= 0;
-                const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-                const long long prow = static_cast<long long>(valid ? e : 0) * p.Hq +
-                                       static_cast<long long>(hk) * G + g;
-                __nv_bfloat16 *dst = p.part_o + prow * D;
-#pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem_o + lane_addr + cc * 32, v);
-                    tmem_wait_ld();
-                    if (valid) {
-                        const uint64_t il2 = f2_pack(inv_l, inv_l);
-                        uint32_t w[16];
-#pragma unroll
-                        for (int x = 0; x < 16; ++x) {
-                            float a0, a1;
-                            f2_unpack(f2_mul(f2_pack(__uint_as_float(v[2 * x]), __uint_as_float(v[2 * x + 1])), il2), a0, a1);
-                            w[x] = pack_bf16x2(a0, a1);
-                        }
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            *reinterpret_cast<uint4 *>(dst + cc * 32 + q4 * 8) =
-                                make_uint4(w[q4 * 4], w[q4 * 4 + 1], w[q4 * 4 + 2], w[q4 * 4 + 3]);
-                    }
-                }
-                if (valid)
-                    p.part_lse[prow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
-                m_run = -INFINITY;
-                l_run = 0.f;
-                tc_fence_before();
             }
         }
         ++item_n;
-        // both warpgroups done with this item's K/V and Q buffers
+        // both warpgroups done with this item's K/V, Q buffers and table
         if (__syncthreads_or(aborted)) {
             aborted = true;
             break;
