@@ -435,12 +435,371 @@ struct ItemRows {
     int t[kItemTokens];           // query position, or -1
 };
 
+// ===========================================================================
+// Prefill attention, K/V block resident (block <= 128): warp-specialised.
+//   warps 0-3 / 4-7: warpgroups WG0 / WG1.  Each takes alternate 128-row
+//     chunks of the item: gathers Q (cp.async, double-buffered), runs the
+//     softmax (S -> P in tensor memory) and the epilogue (normalised bf16
+//     partial rows staged in shared memory, one bulk copy per token).
+//   warp 8 (one thread): TMA-loads K_j and V_j once per item and issues every
+//     tcgen05.mma for both warpgroups from a non-blocking event loop:
+//       S(w, i)  when Q(w, i) is ready and PV(w, i-1) has completed,
+//       PV(w, i) when P(w, i) is ready.
+//     So S of a warpgroup's next chunk runs on the tensor core while that
+//     warpgroup is in the epilogue of the current one.
+// Tensor memory: WG w owns columns [256w, 256w+256): S/P at +0, O at +128.
+// ===========================================================================
+template <int D>
+__global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    AttnParams p) {
+    constexpr int DREG = D / 64;
+    constexpr uint32_t QBYTES = DREG * kRegionBytes + 2048;  // Q tile + staging room
+    constexpr int PPR = D / 8;
+    const int NK = p.NK;
+    const uint32_t kv_tile = static_cast<uint32_t>(NK) * 128u * DREG;
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = align1024(smem_raw);
+    unsigned char *kv_s = base;                        // K tile, V tile
+    unsigned char *q_s = kv_s + 2 * kv_tile;           // [wg][buf]
+    ItemRows *tab = reinterpret_cast<ItemRows *>(q_s + 4 * QBYTES);
+    uint64_t *kvfull = reinterpret_cast<uint64_t *>(tab + 1);
+    uint64_t *bar_s = kvfull + 1;    // [wg] S(w, i) complete
+    uint64_t *bar_o = kvfull + 3;    // [wg] PV(w, i) complete
+    uint64_t *q_ready = kvfull + 5;  // [wg] Q(w, i) in shared memory
+    uint64_t *p_ready = kvfull + 7;  // [wg] P(w, i) in tensor memory
+    int *sh_item = reinterpret_cast<int *>(kvfull + 9);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sh_item + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid & 31;
+    const bool is_mma = warp == 8;
+    const int wg = is_mma ? 0 : (warp >> 2), wtid = tid & 127;
+    const uint32_t wg_bar = 1 + wg;
+    if (tid == 0) {
+        mbar_init(kvfull, 1);
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(bar_s + w, 1);
+            mbar_init(bar_o + w, 1);
+            mbar_init(q_ready + w, 1);
+            mbar_init(p_ready + w, 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_s = tmem_base + static_cast<uint32_t>(wg * 256);
+    const uint32_t tmem_o = tmem_s + 128;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+
+    const int n_items = p.counters[0];
+    const int total = n_items * p.Hkv;
+    const int G = p.G, TOK = p.TOK, K = p.K;
+    const int row = wtid;
+    const int tok = row >> p.log2G, g = row & (G - 1);
+
+    // warpgroup-side phase counters, and the MMA thread's per-warpgroup ones
+    uint32_t s_n = 0, o_n = 0, item_n = 0;
+    uint32_t mq[2] = {0, 0}, mp[2] = {0, 0};
+    int kv_armed = -1;
+    bool aborted = false;
+    int cur_j = 0, cur_hk = 0;
+
+    auto gather = [&](int buf, int c) {
+        unsigned char *dst_base = q_s + (wg * 2 + buf) * QBYTES;
+#pragma unroll 4
+        for (int pc = wtid; pc < 128 * PPR; pc += 128) {
+            const int r = pc / PPR, cc = pc % PPR;
+            const int ti = c * TOK + (r >> p.log2G);
+            const bool ok = tab->t[ti] >= 0;
+            const __nv_bfloat16 *src = p.q + (ok ? tab->qoff[ti] + (r & (G - 1)) * D + cc * 8 : 0);
+            cp_async_16_ca(dst_base + (cc / 8) * kRegionBytes + sw128_offset(r, cc % 8), src,
+                           ok ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+
+    auto wait_wg = [&](uint64_t *bar, uint32_t parity) -> bool {
+        bool ok = true;
+        if (wtid == 0) ok = mbar_wait(bar, parity, abort_flag, p.status);
+        return !named_barrier_or(wg_bar, 128, !ok || *abort_flag);
+    };
+
+    // softmax of this thread's row in two passes over tensor memory, 32
+    // columns at a time (max, then P = 2^(s*c - m) written over the columns
+    // of S already read); keeps 32 scores live instead of 128
+    auto softmax_tile = [&](int c, float &m_run, float &l_run) {
+        tc_fence_after();
+        const int t = tab->t[c * TOK + tok];
+        const int lim = t - cur_j * p.block;  // valid key columns: <= lim
+        const bool masked = lim < NK - 1;
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        for (int cc = 0; cc < NK / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tmem_s + lane_addr + cc * 32, v);
+            tmem_wait_ld();
+            float sv[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+                sv[x] = (masked && cc * 32 + x > lim) ? -INFINITY : __uint_as_float(v[x]);
+#pragma unroll
+            for (int x = 0; x < 32; x += 8) {
+                m4[0] = fmax3(m4[0], sv[x], sv[x + 1]);
+                m4[1] = fmax3(m4[1], sv[x + 2], sv[x + 3]);
+                m4[2] = fmax3(m4[2], sv[x + 4], sv[x + 5]);
+                m4[3] = fmax3(m4[3], sv[x + 6], sv[x + 7]);
+            }
+        }
+        m_run = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * p.scale_log2;
+        const float mref = m_run == -INFINITY ? 0.f : m_run;
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(-mref, -mref);
+        uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
+        for (int cc = 0; cc < NK / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tmem_s + lane_addr + cc * 32, v);
+            tmem_wait_ld();
+            uint32_t w16[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                const float s0 = (masked && cc * 32 + 2 * x > lim) ? -INFINITY : __uint_as_float(v[2 * x]);
+                const float s1 = (masked && cc * 32 + 2 * x + 1 > lim) ? -INFINITY : __uint_as_float(v[2 * x + 1]);
+                float a0, a1;
+                f2_unpack(f2_fma(f2_pack(s0, s1), sc2, nm2), a0, a1);
+                const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+                if (x & 1)
+                    ls2b = f2_add(ls2b, f2_pack(p0, p1));
+                else
+                    ls2a = f2_add(ls2a, f2_pack(p0, p1));
+                w16[x] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tmem_s + lane_addr + cc * 16, w16);
+        }
+        float la0, la1, lb0, lb1;
+        f2_unpack(ls2a, la0, la1);
+        f2_unpack(ls2b, lb0, lb1);
+        l_run = (la0 + la1) + (lb0 + lb1);
+        tmem_wait_st();
+        tc_fence_before();
+    };
+
+    // normalised bf16 partial rows staged token-major (16-byte pad per token)
+    // in `stage`, one bulk copy per token; lse stored directly
+    auto epilogue = [&](int c, float m_run, float l_run, unsigned char *stage) {
+        tc_fence_after();
+        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        const uint64_t il2 = f2_pack(inv_l, inv_l);
+        const uint32_t tok_bytes = static_cast<uint32_t>(G * D * 2 + 16);
+        unsigned char *srow = stage + tok * tok_bytes + g * (D * 2);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tmem_o + lane_addr + cc * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                uint32_t w[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    float a0, a1;
+                    f2_unpack(f2_mul(f2_pack(__uint_as_float(v[q4 * 8 + 2 * x]), __uint_as_float(v[q4 * 8 + 2 * x + 1])), il2), a0, a1);
+                    w[x] = pack_bf16x2(a0, a1);
+                }
+                *reinterpret_cast<uint4 *>(srow + (cc * 4 + q4) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        tc_fence_before();
+        const int e = tab->entry[c * TOK + tok];
+        if (e >= 0) {
+            const long long prow = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G + g;
+            p.part_lse[prow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
+        }
+        fence_proxy_async_smem();
+        if (G <= 32)
+            __syncwarp();
+        else
+            named_barrier(wg_bar, 128);
+        if (g == 0 && e >= 0) {
+            const long long prow0 = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G;
+            bulk_store(p.part_o + prow0 * D, stage + tok * tok_bytes, static_cast<uint32_t>(G * D * 2));
+            bulk_commit();
+        }
+    };
+
+    while (true) {
+        if (tid == 0) *sh_item = atomicAdd(p.counters + 1, 1);
+        __syncthreads();
+        const int w = *sh_item;
+        if (w >= total || *abort_flag) break;
+        const int hk = w / n_items;
+        const AttnItem item = p.items[w - hk * n_items];
+        const int b = item.pair / p.N, j = item.pair - b * p.N;
+        cur_j = j;
+        cur_hk = hk;
+        const int list_base = p.row_ptr[item.pair] + item.start;
+        const int ntok = item.count;
+        const int n_chunks = (ntok + TOK - 1) / TOK;
+
+        if (is_mma && lane == 0) {
+            mbar_arrive_expect_tx(kvfull, 2 * kv_tile);
+            kv_armed = static_cast<int>(item_n & 1);
+            const int z = b * p.T + j * p.block;
+            for (int r = 0; r < DREG; ++r) {
+                tma_load_3d(kv_s + r * NK * 128, &tm_k, kvfull, r * 64, hk, z);
+                tma_load_3d(kv_s + kv_tile + r * NK * 128, &tm_v, kvfull, r * 64, hk, z);
+            }
+        }
+        for (int i = tid; i < n_chunks * TOK; i += blockDim.x) {
+            int e = -1, t = -1;
+            long long qoff = 0;
+            if (i < ntok) {
+                e = p.entries[list_base + i];
+                const int qrow = e >= 0 ? e / K : -1;
+                const int bi = qrow >= 0 ? qrow / p.n_q : -1;
+                if (e < 0 || bi != b) {
+                    atomicOr(p.status, kDevBadIds);
+                    e = -1;
+                } else {
+                    t = p.T - p.n_q + (qrow - bi * p.n_q);
+                    qoff = (static_cast<long long>(qrow) * p.Hq + static_cast<long long>(hk) * G) * D;
+                }
+            }
+            tab->entry[i] = e;
+            tab->t[i] = t;
+            tab->qoff[i] = qoff;
+        }
+        __syncthreads();
+
+        if (is_mma) {
+            if (lane == 0) {
+                // ---- MMA issuer: event loop over both warpgroups' chunks
+                const int nw[2] = {(n_chunks + 1) / 2, n_chunks / 2};
+                int iw[2] = {0, 0}, act[2] = {0, 0};  // act: 0 = S next, 1 = PV next
+                bool ok = mbar_wait(kvfull, item_n & 1, abort_flag, p.status);
+                kv_armed = -1;
+                const uint32_t idesc_s = idesc_bf16_f32(128, NK, false);
+                const uint32_t idesc_o = idesc_bf16_f32(128, D, true);
+                const uint32_t ka = smem_addr(kv_s), va = smem_addr(kv_s + kv_tile);
+                uint64_t t0 = global_timer_ns();
+                while (ok && (iw[0] < nw[0] || iw[1] < nw[1])) {
+                    bool progress = false;
+                    for (int x = 0; x < 2; ++x) {
+                        if (iw[x] >= nw[x]) continue;
+                        const uint32_t ts = tmem_base + static_cast<uint32_t>(x * 256);
+                        if (act[x] == 0) {
+                            if (!mbar_test(q_ready + x, mq[x] & 1)) continue;
+                            if (iw[x] > 0 && !mbar_test(bar_o + x, (mp[x] - 1) & 1)) continue;
+                            tc_fence_after();
+                            const uint32_t qa = smem_addr(q_s + (x * 2 + (iw[x] & 1)) * QBYTES);
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                umma_bf16(ts, sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
+                                          sdesc_sw128(ka + (kk / 4) * NK * 128 + (kk % 4) * 32, 16, 1024),
+                                          idesc_s, kk > 0 ? 1u : 0u);
+                            umma_commit(bar_s + x);
+                            ++mq[x];
+                            act[x] = 1;
+                            progress = true;
+                        } else {
+                            if (!mbar_test(p_ready + x, mp[x] & 1)) continue;
+                            tc_fence_after();
+                            for (int kk = 0; kk < NK / 16; ++kk)
+                                umma_bf16_tmem_a(ts + 128, ts + kk * 8,
+                                                 sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
+                                                 idesc_o, kk > 0 ? 1u : 0u);
+                            umma_commit(bar_o + x);
+                            ++mp[x];
+                            act[x] = 0;
+                            ++iw[x];
+                            progress = true;
+                        }
+                    }
+                    if (progress) {
+                        t0 = global_timer_ns();
+                    } else if (*abort_flag) {
+                        ok = false;
+                    } else if (global_timer_ns() - t0 > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        atomicOr(p.status, kDevTimeout);
+                        ok = false;
+                    }
+                }
+                if (!ok) aborted = true;
+            }
+        } else {
+            // ---- warpgroup: its chunks c = wg, wg + 2, ...
+            const int n = n_chunks > wg ? (n_chunks - wg + 1) / 2 : 0;
+            if (n > 0) {
+                gather(0, wg);
+                if (n > 1) {
+                    gather(1, wg + 2);
+                    cp_async_wait_1();
+                } else {
+                    cp_async_wait_all();
+                }
+                fence_proxy_async_smem();
+                named_barrier(wg_bar, 128);
+                if (wtid == 0) mbar_arrive(q_ready + wg);
+            }
+            for (int ci = 0; ci < n; ++ci) {
+                const int c = wg + 2 * ci, buf = ci & 1;
+                if (!wait_wg(bar_s + wg, s_n & 1)) { aborted = true; break; }
+                ++s_n;
+                float m_run, l_run;
+                softmax_tile(c, m_run, l_run);
+                named_barrier(wg_bar, 128);
+                if (wtid == 0) mbar_arrive(p_ready + wg);
+                if (ci + 1 < n) {
+                    // Q of the next chunk (gathered a chunk ago) -> MMA thread
+                    cp_async_wait_all();
+                    fence_proxy_async_smem();
+                    named_barrier(wg_bar, 128);
+                    if (wtid == 0) mbar_arrive(q_ready + wg);
+                }
+                if (!wait_wg(bar_o + wg, o_n & 1)) { aborted = true; break; }
+                ++o_n;
+                epilogue(c, m_run, l_run, q_s + (wg * 2 + buf) * QBYTES);
+                if (ci + 2 < n) {
+                    bulk_wait_read_all();
+                    named_barrier(wg_bar, 128);
+                    gather(buf, c + 4);
+                }
+            }
+            bulk_wait_read_all();
+        }
+        ++item_n;
+        if (__syncthreads_or(aborted)) {
+            aborted = true;
+            break;
+        }
+    }
+    __syncthreads();
+    if (aborted && is_mma && lane == 0 && kv_armed >= 0) mbar_drain(kvfull, static_cast<uint32_t>(kv_armed));
+    cp_async_wait_all();
+    bulk_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem_base, 512);
+}
+
 template <int D>
 __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     AttnParams p) {
     constexpr int DREG = D / 64;                 // swizzled regions per Q row block
-    constexpr uint32_t QBYTES = DREG * kRegionBytes;
+    // Q tile (DREG swizzled regions) plus room for the epilogue's staging
+    // layout, which pads every token by 16 bytes (at most 128 tokens)
+    constexpr uint32_t QBYTES = DREG * kRegionBytes + 2048;
     constexpr int PPR = D / 8;                   // 16-byte pieces per Q row
     const int NK = p.NK;
     const uint32_t kv_tile = static_cast<uint32_t>(NK) * 128u * DREG;  // one of K or V
@@ -718,17 +1077,18 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
     };
 
     // Normalised bf16 partial and its natural-log lse for chunk c.  Each
-    // thread packs its row and writes it to `stage` (the chunk's Q buffer,
-    // dead once S is done) with 16-byte pieces XOR-swizzled by the row; the
-    // warpgroup then reads the tile back two rows per warp instruction and
-    // stores whole rows (the G rows of a token are contiguous in the
-    // partials), so every global store instruction writes 512 contiguous
-    // bytes.
+    // thread packs its row into `stage` (the chunk's Q buffer, dead once S is
+    // done) in a token-major layout padded by 16 bytes per token (so the
+    // rows a warp writes at once spread over all banks); the first thread of
+    // each token then writes the token's G contiguous head rows of the
+    // partials with one bulk copy.  Callers wait for the copies' reads
+    // (bulk_wait_read_all) before reusing `stage`.
     auto epilogue = [&](int c, float m_run, float l_run, unsigned char *stage) {
         tc_fence_after();
         const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
         const uint64_t il2 = f2_pack(inv_l, inv_l);
-        unsigned char *srow = stage + row * (D * 2);
+        const uint32_t tok_bytes = static_cast<uint32_t>(G * D * 2 + 16);
+        unsigned char *srow = stage + tok * tok_bytes + g * (D * 2);
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t v[32];
@@ -743,31 +1103,24 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                     f2_unpack(f2_mul(f2_pack(__uint_as_float(v[q4 * 8 + 2 * x]), __uint_as_float(v[q4 * 8 + 2 * x + 1])), il2), a0, a1);
                     w[x] = pack_bf16x2(a0, a1);
                 }
-                const int piece = cc * 4 + q4;
-                *reinterpret_cast<uint4 *>(srow + ((piece ^ (row & (PPR - 1))) << 4)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(srow + (cc * 4 + q4) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
+        tc_fence_before();
         const int e = tab->entry[c * TOK + tok];
         if (e >= 0) {
             const long long prow = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G + g;
             p.part_lse[prow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
         }
-        tc_fence_before();
-        named_barrier(wg_bar, 128);
-        // coalesced copy-out: lane -> (row r = base + lane / PPR, piece lane % PPR)
-        constexpr int RPI = 32 / PPR;  // rows per warp instruction
-        const int wl = wtid & 31, wq = wtid >> 5;
-        const int piece = wl % PPR;
-#pragma unroll 4
-        for (int it = 0; it < 32 / RPI; ++it) {
-            const int r = wq * 32 + it * RPI + wl / PPR;
-            const int er = tab->entry[c * TOK + (r >> p.log2G)];
-            const uint4 u = *reinterpret_cast<const uint4 *>(stage + r * (D * 2) + ((piece ^ (r & (PPR - 1))) << 4));
-            if (er >= 0) {
-                const long long prow = static_cast<long long>(er) * p.Hq + static_cast<long long>(cur_hk) * G + (r & (G - 1));
-                *reinterpret_cast<uint4 *>(p.part_o + prow * D + piece * 8) = u;
-            }
+        fence_proxy_async_smem();
+        if (G <= 32)
+            __syncwarp();  // a token's rows all belong to this warp
+        else
+            named_barrier(wg_bar, 128);
+        if (g == 0 && e >= 0) {
+            const long long prow0 = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G;
+            bulk_store(p.part_o + prow0 * D, stage + tok * tok_bytes, static_cast<uint32_t>(G * D * 2));
+            bulk_commit();
         }
     };
 
@@ -828,8 +1181,13 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                     named_barrier(wg_bar, 128);
                 }
                 issue_s(buf, kd);
-                // next chunk's Q into the other buffer (its S finished a chunk ago)
-                if (ci + 1 < n) gather(buf ^ 1, c + 2);
+                // next chunk's Q into the other buffer: its S finished a chunk ago
+                // and its staged partial has been read by the bulk copies
+                if (ci + 1 < n) {
+                    bulk_wait_read_all();
+                    named_barrier(wg_bar, 128);
+                    gather(buf ^ 1, c + 2);
+                }
                 if (!wait_wg(bar_s + wg, s_n & 1)) { aborted = true; break; }
                 ++s_n;
                 float m_run, l_run;
@@ -852,7 +1210,8 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                 const int c = wg + 2 * ci;
                 const bool active = c < n_chunks;
                 if (kt == 0 && active && ci > 0) {
-                    named_barrier(wg_bar, 128);  // staged partial of the previous chunk read out
+                    bulk_wait_read_all();  // staged partial of the previous chunk read out
+                    named_barrier(wg_bar, 128);
                     gather(0, c);
                 }
                 if (kt == 0) cp_async_wait_all();
@@ -885,6 +1244,7 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
             }
         }
         ++item_n;
+        bulk_wait_read_all();  // staged partials read before the buffers are reused
         // both warpgroups done with this item's K/V, Q buffers and table
         if (__syncthreads_or(aborted)) {
             aborted = true;
@@ -897,6 +1257,7 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
             if (armed_parity[s2] >= 0) mbar_drain(kvfull + s2, static_cast<uint32_t>(armed_parity[s2]));
     }
     cp_async_wait_all();
+    bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(*tmem_slot, 512);
@@ -962,8 +1323,8 @@ size_t prefill_attn_smem_bytes(const Shape &sh) {
     const int KVST = NS > 1 ? 2 : 1;
     const int QBUF = NS > 1 ? 1 : 2;
     const size_t kv_tile = static_cast<size_t>(NK) * 128 * (sh.d / 64);
-    const size_t q = static_cast<size_t>(sh.d / 64) * kRegionBytes;
-    return 1024 + KVST * 2 * kv_tile + 2 * QBUF * q + sizeof(ItemRows) + 64 + 32;
+    const size_t q = static_cast<size_t>(sh.d / 64) * kRegionBytes + 2048;
+    return 1024 + KVST * 2 * kv_tile + 2 * QBUF * q + sizeof(ItemRows) + 128 + 32;
 }
 
 int prefill_attn_rows_per_item(int G) {
@@ -1000,15 +1361,20 @@ cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const 
     while ((1 << ap.log2G) < sh.G) ++ap.log2G;
     ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(sh.d));
     const size_t smem = prefill_attn_smem_bytes(sh);
-    if (sh.d == 128) {
-        cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-        prefill_attn_kernel<128><<<num_sms, 256, smem, st>>>(tm_k, tm_v, ap);
+#define MSA_LAUNCH(KERNEL, THREADS)                                                              \
+    do {                                                                                         \
+        cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize,                \
+                             static_cast<int>(smem));                                            \
+        KERNEL<<<num_sms, THREADS, smem, st>>>(tm_k, tm_v, ap);                                  \
+    } while (0)
+    if (ap.NS == 1) {
+        if (sh.d == 128) MSA_LAUNCH(prefill_attn_resident_kernel<128>, 288);
+        else MSA_LAUNCH(prefill_attn_resident_kernel<64>, 288);
     } else {
-        cudaFuncSetAttribute(prefill_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-        prefill_attn_kernel<64><<<num_sms, 256, smem, st>>>(tm_k, tm_v, ap);
+        if (sh.d == 128) MSA_LAUNCH(prefill_attn_kernel<128>, 256);
+        else MSA_LAUNCH(prefill_attn_kernel<64>, 256);
     }
+#undef MSA_LAUNCH
     return cudaGetLastError();
 }
 
