@@ -65,48 +65,59 @@ __device__ __forceinline__ uint4 ld_stream16(const uint4 *p) {
 template <int D_IDX>
 __global__ void __launch_bounds__(256) decode_index_scan_kernel(
     const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16 *__restrict__ k_idx,
-    float *__restrict__ block_scores, int T, int block, int own, int N) {
+    float *__restrict__ block_scores, int Bt, int T, int block, int own, int N, int rw, int bpc) {
+    // rw: rows per warp (a warp's rows lie in one block); bpc: blocks per CTA
     constexpr int LPR = D_IDX / 8;  // lanes per key row
     constexpr int RPL = 32 / LPR;   // key rows per warp load
     constexpr int UNR = 16;         // loads in flight per warp
     __shared__ float wmax[8];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = lane / LPR, part = lane % LPR;
-    const int b = blockIdx.x / own, j = blockIdx.x % own;
-    float qv[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4 *>(q_idx + static_cast<long long>(b) * D_IDX + part * 8), qv);
-    const uint4 *base = reinterpret_cast<const uint4 *>(
-        k_idx + (static_cast<long long>(b) * T + static_cast<long long>(j) * block) * D_IDX);
-    // rows of this warp: r = (warp + 8 * it) * RPL + sub
-    const int groups = block / RPL;  // row groups of RPL rows
+    const int wpb = 8 / bpc;                         // warps per block
+    const long long item = static_cast<long long>(blockIdx.x) * bpc + warp / wpb;
+    const bool active = item < static_cast<long long>(Bt) * own;
     float best = -FLT_MAX;
-    for (int g0 = warp; g0 < groups; g0 += 8 * UNR) {
-        uint4 ku[UNR];
+    if (active) {
+        const int b = static_cast<int>(item / own), j = static_cast<int>(item % own);
+        float qv[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(q_idx + static_cast<long long>(b) * D_IDX + part * 8), qv);
+        // the wpb warps of block j interleave over its row groups
+        const int wi = warp % wpb;
+        const uint4 *base = reinterpret_cast<const uint4 *>(
+            k_idx + (static_cast<long long>(b) * T + static_cast<long long>(j) * block) * D_IDX);
+        const int groups = rw / RPL;  // row groups per warp
+        for (int g0 = 0; g0 < groups; g0 += UNR) {
+            uint4 ku[UNR];
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const int gi = g0 + 8 * u;
-            ku[u] = gi < groups ? ld_stream16(base + (gi * RPL + sub) * LPR + part) : make_uint4(0, 0, 0, 0);
+            for (int u = 0; u < UNR; ++u) {
+                const int gi = wi + wpb * (g0 + u);
+                ku[u] = g0 + u < groups ? ld_stream16(base + (gi * RPL + sub) * LPR + part)
+                                        : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                float kf[8];
+                bf16x8_to_f32(ku[u], kf);
+                float sc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sc = fmaf(qv[e], kf[e], sc);
+#pragma unroll
+                for (int o = LPR / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xFFFFFFFFu, sc, o);
+                if (g0 + u < groups) best = fmaxf(best, sc);
+            }
         }
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            float kf[8];
-            bf16x8_to_f32(ku[u], kf);
-            float s = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) s = fmaf(qv[e], kf[e], s);
-#pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-            if (g0 + 8 * u < groups) best = fmaxf(best, s);
-        }
+        for (int o = LPR; o < 32; o <<= 1) best = fmaxf(best, __shfl_xor_sync(0xFFFFFFFFu, best, o));
     }
-#pragma unroll
-    for (int o = LPR; o < 32; o <<= 1) best = fmaxf(best, __shfl_xor_sync(0xFFFFFFFFu, best, o));
     if (lane == 0) wmax[warp] = best;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        float m = wmax[0];
-        for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
-        block_scores[static_cast<long long>(b) * N + j] = m;
+    if (threadIdx.x < bpc) {
+        const long long it = static_cast<long long>(blockIdx.x) * bpc + threadIdx.x;
+        if (it < static_cast<long long>(Bt) * own) {
+            float m = -FLT_MAX;
+            for (int w = threadIdx.x * wpb; w < (threadIdx.x + 1) * wpb; ++w) m = fmaxf(m, wmax[w]);
+            block_scores[(it / own) * N + it % own] = m;
+        }
     }
 }
 
@@ -181,39 +192,63 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
 }
 
 // ------------------------------------------------------------------------
-// Split-K decode attention.  One CTA of 128 threads per (b, kv head, slot,
-// split of kDecodeKeys keys).  K/V rows are staged in shared memory by
-// 16-byte cp.async (coalesced 2*d-byte rows); the G query heads share them.
-// Scores: thread (key = tid/2, half = tid%2) holds its half K row in
-// registers and reads q (pre-scaled, fp32) as broadcast float4; the two
-// halves are summed by a shuffle.  Softmax in the log2 domain, one warp per
-// head.  PV: thread per output column (and key half when d = 64), p read as
-// float4 over heads.  Writes a normalised fp32 partial and its natural-log
-// lse (-inf when the split has no key).
+// Split-K decode attention on mma.sync (m16n8k16, bf16 in, fp32 accumulate).
+// One CTA of 4 warps per (b, kv head, slot, split of kDecodeKeys keys); warp
+// w owns keys [16w, 16w+16) of the split.  K/V rows are staged in shared
+// memory by 16-byte cp.async (coalesced 2*d-byte rows, padded by 16 bytes so
+// ldmatrix reads are conflict-free; rows past the split's end are zero).  The
+// G query heads of the kv head are processed 16 at a time (heads past G are
+// zero rows): S = Q K^T (16 heads x 16 keys), softmax per head in the log2
+// domain, O = P V with P taken straight from the S fragments; the four
+// warps' partials are merged in shared memory.  Writes a normalised fp32
+// partial and its natural-log lse (-inf when the split has no key).
 // ------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) decode_attn_kernel(
     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
     const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ ids,
     float *__restrict__ part_o, float *__restrict__ part_lse, int T, int Hq, int Hkv, int block,
     int K, int S, int N, float scale_log2, int *__restrict__ status) {
-    constexpr int KS = kDecodeKeys;
-    constexpr int KSTR = D + 8;       // padded K row (bf16) to spread banks
-    constexpr int HALF = D / 2;       // elements of a half row
-    constexpr int NH = 128 / D;       // key halves in the PV phase
+    constexpr int KS = kDecodeKeys;  // 64 keys = 4 warps x 16
+    constexpr int STR = D + 8;       // padded row (bf16 elements)
+    constexpr int PIECES = D / 8;    // 16-byte pieces per row
+    constexpr int NT = D / 8;        // n-tiles of the PV product
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int G = Hq / Hkv;
-    const int GP = (G + 3) & ~3;      // heads padded to a float4
-    float *qs = reinterpret_cast<float *>(smem_raw);   // [G][D]
-    float *ps = qs + G * D;                             // [KS][GP]
-    float *ms = ps + KS * GP;                           // [G]
-    float *ls = ms + G;                                 // [G]
-    float *red = ls + G;                                // [NH-1][G][D] (d = 64 only)
-    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(
-        (reinterpret_cast<uintptr_t>(red + (NH - 1) * G * D) + 15) & ~static_cast<uintptr_t>(15));
-    __nv_bfloat16 *Vs = Ks + KS * KSTR;                 // [KS][D]
+    __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(smem_raw);  // [KS][STR]
+    __nv_bfloat16 *Vs = Ks + KS * STR;                                  // [KS][STR]
+    __nv_bfloat16 *Qs = Vs + KS * STR;                                  // [16][STR]
+    __nv_bfloat16 *Ps = Qs + 16 * STR;                                  // [16][KS + 8]
+    float *mw = reinterpret_cast<float *>(Ps + 16 * (KS + 8));          // [4][16]
+    float *lw = mw + 64;                                                // [4][16]
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gq = lane >> 2, tq = lane & 3;  // mma fragment coordinates
     int idx = blockIdx.x;
     const int sp = idx % S;
     idx /= S;
@@ -221,6 +256,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     idx /= K;
     const int hk = idx % Hkv;
     const int b = idx / Hkv;
+    const int G = Hq / Hkv;
     const long long prow = (static_cast<long long>(b) * K + s) * S + sp;  // partial row
     const int t = T - 1;
     const int j = ids[static_cast<long long>(b) * K + s];
@@ -241,136 +277,143 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
         for (int g = tid; g < G; g += blockDim.x) part_lse[prow * Hq + hk * G + g] = -INFINITY;
         return;
     }
-    constexpr int PIECES = D / 8;  // 16-byte pieces per row
+    // stage K and V rows (zero past nk)
     const __nv_bfloat16 *kbase = k + ((static_cast<long long>(b) * T + k0) * Hkv + hk) * D;
     const __nv_bfloat16 *vbase = v + ((static_cast<long long>(b) * T + k0) * Hkv + hk) * D;
-    for (int e = tid; e < nk * PIECES; e += blockDim.x) {
+    for (int e = tid; e < KS * PIECES; e += blockDim.x) {
         const int r = e / PIECES, c = e % PIECES;
-        const long long goff = static_cast<long long>(r) * Hkv * D + c * 8;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                         static_cast<uint32_t>(__cvta_generic_to_shared(Ks + r * KSTR + c * 8))),
-                     "l"(kbase + goff)
+        const bool ok = r < nk;
+        const long long goff = ok ? static_cast<long long>(r) * Hkv * D + c * 8 : 0;
+        const uint32_t bytes = ok ? 16u : 0u;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                         static_cast<uint32_t>(__cvta_generic_to_shared(Ks + r * STR + c * 8))),
+                     "l"(kbase + goff), "r"(bytes)
                      : "memory");
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                         static_cast<uint32_t>(__cvta_generic_to_shared(Vs + r * D + c * 8))),
-                     "l"(vbase + goff)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                         static_cast<uint32_t>(__cvta_generic_to_shared(Vs + r * STR + c * 8))),
+                     "l"(vbase + goff), "r"(bytes)
                      : "memory");
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    const __nv_bfloat16 *qrow = q + (static_cast<long long>(b) * Hq + hk * G) * D;
-    for (int e = tid; e < G * D; e += blockDim.x) qs[e] = __bfloat162float(qrow[e]) * scale_log2;
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncthreads();
+    const int key0 = warp * 16;  // this warp's keys
 
-    // ---- scores: ps[key][g] (log2 domain)
-    {
-        const int key = tid >> 1, half = tid & 1;
-        const bool kv_ok = key < nk;
-        uint4 kr[HALF / 8];
+    for (int g0 = 0; g0 < G; g0 += 16) {
+        // Q rows g0..g0+15 of this kv head group (zero past G), bf16
+        const __nv_bfloat16 *qrow = q + (static_cast<long long>(b) * Hq + hk * G + g0) * D;
+        for (int e = tid; e < 16 * PIECES; e += blockDim.x) {
+            const int r = e / PIECES, c = e % PIECES;
+            uint4 u = make_uint4(0, 0, 0, 0);
+            if (g0 + r < G) u = *reinterpret_cast<const uint4 *>(qrow + r * D + c * 8);
+            *reinterpret_cast<uint4 *>(Qs + r * STR + c * 8) = u;
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+
+        // ---- S = Q K^T: 16 heads x 16 keys (two n-tiles of 8 keys)
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const int mi = lane >> 3, ri = lane & 7;
 #pragma unroll
-        for (int c = 0; c < HALF / 8; ++c)
-            kr[c] = kv_ok ? *reinterpret_cast<const uint4 *>(Ks + key * KSTR + half * HALF + c * 8)
-                          : make_uint4(0, 0, 0, 0);
-        for (int g0 = 0; g0 < G; g0 += 8) {
-            float acc[8];
+        for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t af[4], bf[4];
+            ldmatrix_x4(af, Qs + ((mi & 1) * 8 + ri) * STR + kk * 16 + (mi >> 1) * 8);
+            ldmatrix_x4(bf, Ks + (key0 + (mi >> 1) * 8 + ri) * STR + kk * 16 + (mi & 1) * 8);
+            mma_bf16_16816(acc[0], af, bf[0], bf[1]);
+            mma_bf16_16816(acc[1], af, bf[2], bf[3]);
+        }
+        // ---- row max over the 64 keys (per-warp partials through shared memory)
+        float x[2][4];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) acc[x] = 0.f;
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int c = 0; c < HALF / 8; ++c) {
-                float kf[8];
-                bf16x8_to_f32(kr[c], kf);
-#pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    if (g0 + x < G) {
-                        const float4 *qp = reinterpret_cast<const float4 *>(qs + (g0 + x) * D + half * HALF + c * 8);
-                        const float4 qa = qp[0], qb = qp[1];
-                        acc[x] = fmaf(qa.x, kf[0], acc[x]);
-                        acc[x] = fmaf(qa.y, kf[1], acc[x]);
-                        acc[x] = fmaf(qa.z, kf[2], acc[x]);
-                        acc[x] = fmaf(qa.w, kf[3], acc[x]);
-                        acc[x] = fmaf(qb.x, kf[4], acc[x]);
-                        acc[x] = fmaf(qb.y, kf[5], acc[x]);
-                        acc[x] = fmaf(qb.z, kf[6], acc[x]);
-                        acc[x] = fmaf(qb.w, kf[7], acc[x]);
-                    }
-                }
+            for (int e = 0; e < 4; ++e) {
+                const int key = key0 + nt * 8 + 2 * tq + (e & 1);
+                x[nt][e] = key < nk ? acc[nt][e] * scale_log2 : -INFINITY;
             }
+        float m0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+        float m1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
 #pragma unroll
-            for (int x = 0; x < 8; ++x) acc[x] += __shfl_xor_sync(0xFFFFFFFFu, acc[x], 1);
-            if (half == 0) {
+        for (int o = 1; o < 4; o <<= 1) {
+            m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, o));
+            m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, o));
+        }
+        if (tq == 0) {
+            mw[warp * 16 + gq] = m0;
+            mw[warp * 16 + gq + 8] = m1;
+        }
+        __syncthreads();
+        float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
-                for (int x = 0; x < 8; ++x)
-                    if (g0 + x < G) ps[key * GP + g0 + x] = kv_ok ? acc[x] : -INFINITY;
+        for (int w = 0; w < 4; ++w) {
+            M0 = fmaxf(M0, mw[w * 16 + gq]);
+            M1 = fmaxf(M1, mw[w * 16 + gq + 8]);
+        }
+        // key 0 of the split is always valid, so M0 and M1 are finite
+        float pr[2][4];
+        float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            pr[nt][0] = exp2f(x[nt][0] - M0);
+            pr[nt][1] = exp2f(x[nt][1] - M0);
+            pr[nt][2] = exp2f(x[nt][2] - M1);
+            pr[nt][3] = exp2f(x[nt][3] - M1);
+            l0 += pr[nt][0] + pr[nt][1];
+            l1 += pr[nt][2] + pr[nt][3];
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, o);
+            l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, o);
+        }
+        if (tq == 0) {
+            lw[warp * 16 + gq] = l0;
+            lw[warp * 16 + gq + 8] = l1;
+        }
+        // P (16 heads x 64 keys, bf16) to shared memory, row stride PSTR
+        constexpr int PSTR = KS + 8;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int col = key0 + nt * 8 + 2 * tq;
+            *reinterpret_cast<uint32_t *>(Ps + gq * PSTR + col) = bf16x2_bits(pr[nt][0], pr[nt][1]);
+            *reinterpret_cast<uint32_t *>(Ps + (gq + 8) * PSTR + col) = bf16x2_bits(pr[nt][2], pr[nt][3]);
+        }
+        __syncthreads();
+        // ---- O[:, 32w .. 32w+31] = P V over all 64 keys (4 k-steps x 4 n-tiles)
+        constexpr int CW = D / 4;  // output columns per warp
+        constexpr int NTW = CW / 8;
+        float o[NTW][4];
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KS / 16; ++kk) {
+            uint32_t pa[4];
+            ldmatrix_x4(pa, Ps + ((mi & 1) * 8 + ri) * PSTR + kk * 16 + (mi >> 1) * 8);
+#pragma unroll
+            for (int nt = 0; nt < NTW; nt += 2) {
+                uint32_t vf[4];
+                ldmatrix_x4_trans(vf, Vs + (kk * 16 + (mi & 1) * 8 + ri) * STR + warp * CW + (nt + (mi >> 1)) * 8);
+                mma_bf16_16816(o[nt], pa, vf[0], vf[1]);
+                mma_bf16_16816(o[nt + 1], pa, vf[2], vf[3]);
             }
         }
+        const float L0 = lw[gq] + lw[16 + gq] + lw[32 + gq] + lw[48 + gq];
+        const float L1 = lw[gq + 8] + lw[24 + gq] + lw[40 + gq] + lw[56 + gq];
+        const float i0 = 1.f / L0, i1 = 1.f / L1;
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt) {
+            const int col = warp * CW + nt * 8 + 2 * tq;
+            if (g0 + gq < G)
+                *reinterpret_cast<float2 *>(part_o + (prow * Hq + hk * G + g0 + gq) * D + col) =
+                    make_float2(o[nt][0] * i0, o[nt][1] * i0);
+            if (g0 + gq + 8 < G)
+                *reinterpret_cast<float2 *>(part_o + (prow * Hq + hk * G + g0 + gq + 8) * D + col) =
+                    make_float2(o[nt][2] * i1, o[nt][3] * i1);
+        }
+        if (warp == 0 && tq == 0) {
+            if (g0 + gq < G) part_lse[prow * Hq + hk * G + g0 + gq] = (M0 + log2f(L0)) * kLn2;
+            if (g0 + gq + 8 < G) part_lse[prow * Hq + hk * G + g0 + gq + 8] = (M1 + log2f(L1)) * kLn2;
+        }
+        __syncthreads();
     }
-    __syncthreads();
-    // ---- per-head max and sum (one warp per head), p in place
-    const int warp = tid / 32, lane = tid % 32;
-    for (int g = warp; g < G; g += blockDim.x / 32) {
-        float mx = -INFINITY;
-        for (int key = lane; key < nk; key += 32) mx = fmaxf(mx, ps[key * GP + g]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-        float sum = 0.f;
-        for (int key = lane; key < KS; key += 32) {
-            const float pv = key < nk ? exp2f(ps[key * GP + g] - mx) : 0.f;
-            ps[key * GP + g] = pv;
-            sum += pv;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        if (lane == 0) {
-            ms[g] = mx;
-            ls[g] = sum;
-        }
-    }
-    __syncthreads();
-    // ---- out[g][c] = sum_key p[key][g] * V[key][c] / l[g]
-    {
-        const int c = tid % D, kh = tid / D;  // column, key half (NH halves)
-        const int kb = kh * (KS / NH), ke = min(nk, kb + KS / NH);
-        for (int g0 = 0; g0 < G; g0 += 8) {
-            float acc[8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) acc[x] = 0.f;
-            for (int key = kb; key < ke; ++key) {
-                const float vv = __bfloat162float(Vs[key * D + c]);
-                const float4 pa = *reinterpret_cast<const float4 *>(ps + key * GP + g0);
-                acc[0] = fmaf(pa.x, vv, acc[0]);
-                acc[1] = fmaf(pa.y, vv, acc[1]);
-                acc[2] = fmaf(pa.z, vv, acc[2]);
-                acc[3] = fmaf(pa.w, vv, acc[3]);
-                if (g0 + 4 < GP) {
-                    const float4 pb = *reinterpret_cast<const float4 *>(ps + key * GP + g0 + 4);
-                    acc[4] = fmaf(pb.x, vv, acc[4]);
-                    acc[5] = fmaf(pb.y, vv, acc[5]);
-                    acc[6] = fmaf(pb.z, vv, acc[6]);
-                    acc[7] = fmaf(pb.w, vv, acc[7]);
-                }
-            }
-            if (NH > 1 && kh > 0) {
-#pragma unroll
-                for (int x = 0; x < 8; ++x)
-                    if (g0 + x < G) red[((kh - 1) * G + g0 + x) * D + c] = acc[x];
-            }
-            if (NH > 1) __syncthreads();
-            if (kh == 0) {
-#pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const int g = g0 + x;
-                    if (g < G) {
-                        float a = acc[x];
-                        for (int h2 = 1; h2 < NH; ++h2) a += red[((h2 - 1) * G + g) * D + c];
-                        part_o[(prow * Hq + hk * G + g) * D + c] = a / ls[g];
-                    }
-                }
-            }
-            if (NH > 1) __syncthreads();
-        }
-    }
-    for (int g = tid; g < G; g += blockDim.x)
-        part_lse[prow * Hq + hk * G + g] = (ms[g] + log2f(ls[g])) * kLn2;
 }
 
 // ------------------------------------------------------------------------
@@ -731,15 +774,29 @@ cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k
     (void)num_sms;
     const int own = (sh.T - 1) / sh.block;
     if (own > 0) {
-        const long long grid = static_cast<long long>(sh.Bt) * own;
+        // 8 warps per CTA; a warp scans at most 64 rows of one block; small
+        // blocks are packed several to a CTA
+        int rw, bpc;
+        if (sh.block <= 64) {
+            rw = sh.block;
+            bpc = 8;
+        } else if (sh.block <= 512 && 512 % sh.block == 0) {
+            rw = 64;
+            bpc = 512 / sh.block;
+        } else {
+            rw = sh.block / 8;
+            bpc = 1;
+        }
+        const long long items = static_cast<long long>(sh.Bt) * own;
+        const long long grid = (items + bpc - 1) / bpc;
         const auto *qi = static_cast<const __nv_bfloat16 *>(q_idx);
         const auto *ki = static_cast<const __nv_bfloat16 *>(k_idx);
         if (sh.d_idx == 128)
             decode_index_scan_kernel<128><<<static_cast<unsigned>(grid), 256, 0, st>>>(
-                qi, ki, block_scores, sh.T, sh.block, own, sh.N);
+                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N, rw, bpc);
         else
             decode_index_scan_kernel<64><<<static_cast<unsigned>(grid), 256, 0, st>>>(
-                qi, ki, block_scores, sh.T, sh.block, own, sh.N);
+                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N, rw, bpc);
     }
     return cudaGetLastError();
 }
@@ -752,14 +809,8 @@ cudaError_t launch_decode_select(const Shape &sh, const float *block_scores, int
 }
 
 size_t decode_attn_smem_bytes(const Shape &sh) {
-    const int G = sh.G;
-    const int GP = (G + 3) & ~3;
-    const int NH = 128 / sh.d;
-    size_t f = static_cast<size_t>(G) * sh.d + static_cast<size_t>(kDecodeKeys) * GP + 2 * G +
-               static_cast<size_t>(NH - 1) * G * sh.d;
-    size_t bytes = align_up(f * 4, 16);
-    bytes += static_cast<size_t>(kDecodeKeys) * (sh.d + 8) * 2 + static_cast<size_t>(kDecodeKeys) * sh.d * 2;
-    return bytes;
+    const size_t str = static_cast<size_t>(sh.d) + 8;
+    return (2 * kDecodeKeys + 16) * str * 2 + static_cast<size_t>(16) * (kDecodeKeys + 8) * 2 + 128 * 4;
 }
 
 cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, const void *v,
