@@ -430,7 +430,7 @@ struct AttnParams {
 // built once per item in shared memory.
 constexpr int kItemTokens = 1024;
 struct ItemRows {
-    long long qoff[kItemTokens];  // element offset of the token's head group hk in q
+    int qo16[kItemTokens];        // offset of the token's head group hk in q, 16-byte units (0 if none)
     int entry[kItemTokens];       // list entry = partial row (b*n_q + i)*K + slot, or -1
     int t[kItemTokens];           // query position, or -1
 };
@@ -438,24 +438,32 @@ struct ItemRows {
 // ===========================================================================
 // Prefill attention, K/V block resident (block <= 128): warp-specialised.
 //   warps 0-3 / 4-7: warpgroups WG0 / WG1.  Each takes alternate 128-row
-//     chunks of the item: gathers Q (cp.async, double-buffered), runs the
-//     softmax (S -> P in tensor memory) and the epilogue (normalised bf16
-//     partial rows staged in shared memory, one bulk copy per token).
-//   warp 8 (one thread): TMA-loads K_j and V_j once per item and issues every
-//     tcgen05.mma for both warpgroups from a non-blocking event loop:
-//       S(w, i)  when Q(w, i) is ready and PV(w, i-1) has completed,
-//       PV(w, i) when P(w, i) is ready.
-//     So S of a warpgroup's next chunk runs on the tensor core while that
-//     warpgroup is in the epilogue of the current one.
+//     chunks of the item.  Per chunk: wait for S, softmax (S -> P in tensor
+//     memory), issue PV, wait for it, issue S of its next chunk (which then
+//     runs under the epilogue), epilogue (normalised bf16 partial rows staged
+//     in shared memory, one bulk copy per token).  One elected thread per
+//     warpgroup issues that warpgroup's tcgen05.mma.
+//   warps 8-11: producers.  Thread 0 of them TMA-loads K_j and V_j once per
+//     item; all gather the Q rows of chunks 0, 1, 2, ... into the owning
+//     warpgroup's two Q buffers: rows are loaded into registers (not
+//     allocated in L1) before the buffer is known to be free, then stored in
+//     the 128-byte-swizzled layout.
+// Q readiness and Q-buffer release are mbarriers per (warpgroup, buffer), so
+// no signaller runs two phases ahead of its waiter.
 // Tensor memory: WG w owns columns [256w, 256w+256): S/P at +0, O at +128.
 // ===========================================================================
+constexpr int kResidentThreads = 384;
+
 template <int D>
-__global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
+__global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     AttnParams p) {
     constexpr int DREG = D / 64;
     constexpr uint32_t QBYTES = DREG * kRegionBytes + 2048;  // Q tile + staging room
-    constexpr int PPR = D / 8;
+    constexpr int PPR = D / 8;        // 16-byte pieces per row
+    constexpr int NPROD = 128;        // producer threads (warps 8-11)
+    constexpr int NLD = PPR;          // pieces per producer thread per chunk
+    constexpr int RSTEP = NPROD / PPR;
     const int NK = p.NK;
     const uint32_t kv_tile = static_cast<uint32_t>(NK) * 128u * DREG;
 
@@ -465,25 +473,29 @@ __global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
     unsigned char *q_s = kv_s + 2 * kv_tile;           // [wg][buf]
     ItemRows *tab = reinterpret_cast<ItemRows *>(q_s + 4 * QBYTES);
     uint64_t *kvfull = reinterpret_cast<uint64_t *>(tab + 1);
-    uint64_t *bar_s = kvfull + 1;    // [wg] S(w, i) complete
-    uint64_t *bar_o = kvfull + 3;    // [wg] PV(w, i) complete
-    uint64_t *q_ready = kvfull + 5;  // [wg] Q(w, i) in shared memory
-    uint64_t *p_ready = kvfull + 7;  // [wg] P(w, i) in tensor memory
-    int *sh_item = reinterpret_cast<int *>(kvfull + 9);
+    uint64_t *bar_s = kvfull + 1;     // [wg]      S(w, i) complete
+    uint64_t *bar_o = kvfull + 3;     // [wg]      PV(w, i) complete
+    uint64_t *q_ready = kvfull + 5;   // [wg][buf] Q tile gathered
+    uint64_t *q_free = kvfull + 9;    // [wg][buf] Q buffer released by its warpgroup
+    int *sh_item = reinterpret_cast<int *>(kvfull + 13);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sh_item + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
-    const int tid = threadIdx.x, warp = tid / 32, lane = tid & 31;
-    const bool is_mma = warp == 8;
-    const int wg = is_mma ? 0 : (warp >> 2), wtid = tid & 127;
+    const int tid = threadIdx.x, warp = tid / 32;
+    const bool is_prod = warp >= 8;
+    const int ptid = tid - 256;  // producer thread index
+    const int wg = is_prod ? 0 : (warp >> 2), wtid = tid & 127;
     const uint32_t wg_bar = 1 + wg;
+    constexpr uint32_t kProdBar = 3;
     if (tid == 0) {
         mbar_init(kvfull, 1);
         for (int w = 0; w < 2; ++w) {
             mbar_init(bar_s + w, 1);
             mbar_init(bar_o + w, 1);
-            mbar_init(q_ready + w, 1);
-            mbar_init(p_ready + w, 1);
+            for (int u = 0; u < 2; ++u) {
+                mbar_init(q_ready + 2 * w + u, 1);
+                mbar_init(q_free + 2 * w + u, 1);
+            }
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -508,36 +520,44 @@ __global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
     const int row = wtid;
     const int tok = row >> p.log2G, g = row & (G - 1);
 
-    // warpgroup-side phase counters, and the MMA thread's per-warpgroup ones
-    uint32_t s_n = 0, o_n = 0, item_n = 0;
-    uint32_t mq[2] = {0, 0}, mp[2] = {0, 0};
+    uint32_t s_n = 0, o_n = 0, item_n = 0;   // warpgroup: bar_s / bar_o phases
+    uint32_t qr_n[2] = {0, 0};                // warpgroup: q_ready phases per buffer
+    uint32_t pf[2][2] = {{0, 0}, {0, 0}};     // producers: q_free phases
     int kv_armed = -1;
     bool aborted = false;
     int cur_j = 0, cur_hk = 0;
-
-    auto gather = [&](int buf, int c) {
-        unsigned char *dst_base = q_s + (wg * 2 + buf) * QBYTES;
-#pragma unroll 4
-        for (int pc = wtid; pc < 128 * PPR; pc += 128) {
-            const int r = pc / PPR, cc = pc % PPR;
-            const int ti = c * TOK + (r >> p.log2G);
-            const bool ok = tab->t[ti] >= 0;
-            const __nv_bfloat16 *src = p.q + (ok ? tab->qoff[ti] + (r & (G - 1)) * D + cc * 8 : 0);
-            cp_async_16_ca(dst_base + (cc / 8) * kRegionBytes + sw128_offset(r, cc % 8), src,
-                           ok ? 16u : 0u);
-        }
-        cp_async_commit();
-    };
 
     auto wait_wg = [&](uint64_t *bar, uint32_t parity) -> bool {
         bool ok = true;
         if (wtid == 0) ok = mbar_wait(bar, parity, abort_flag, p.status);
         return !named_barrier_or(wg_bar, 128, !ok || *abort_flag);
     };
+    const uint32_t idesc_s = idesc_bf16_f32(128, NK, false);
+    const uint32_t idesc_o = idesc_bf16_f32(128, D, true);
+    // S = Q K^T for the Q tile in buffer `buf` (elected thread)
+    auto issue_s = [&](int buf) {
+        tc_fence_after();
+        const uint32_t qa = smem_addr(q_s + (wg * 2 + buf) * QBYTES), ka = smem_addr(kv_s);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+            umma_bf16(tmem_s, sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
+                      sdesc_sw128(ka + (kk / 4) * NK * 128 + (kk % 4) * 32, 16, 1024), idesc_s,
+                      kk > 0 ? 1u : 0u);
+        umma_commit(bar_s + wg);
+    };
+    // O = P V with P (bf16) in tensor memory (elected thread)
+    auto issue_pv = [&]() {
+        tc_fence_after();
+        const uint32_t va = smem_addr(kv_s + kv_tile);
+        for (int kk = 0; kk < NK / 16; ++kk)
+            umma_bf16_tmem_a(tmem_o, tmem_s + kk * 8,
+                             sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
+                             idesc_o, kk > 0 ? 1u : 0u);
+        umma_commit(bar_o + wg);
+    };
 
-    // softmax of this thread's row in two passes over tensor memory, 32
-    // columns at a time (max, then P = 2^(s*c - m) written over the columns
-    // of S already read); keeps 32 scores live instead of 128
+    // softmax of this thread's row in two passes over tensor memory: row max,
+    // then P = 2^(s*c - m) as bf16 written over the columns of S already read
     auto softmax_tile = [&](int c, float &m_run, float &l_run) {
         tc_fence_after();
         const int t = tab->t[c * TOK + tok];
@@ -602,9 +622,9 @@ __global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
         const uint32_t tok_bytes = static_cast<uint32_t>(G * D * 2 + 16);
         unsigned char *srow = stage + tok * tok_bytes + g * (D * 2);
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
+        for (int c64 = 0; c64 < D; c64 += 32) {
             uint32_t v[32];
-            tmem_ld32(tmem_o + lane_addr + cc * 32, v);
+            tmem_ld32(tmem_o + lane_addr + c64, v);
             tmem_wait_ld();
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
@@ -615,7 +635,7 @@ __global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
                     f2_unpack(f2_mul(f2_pack(__uint_as_float(v[q4 * 8 + 2 * x]), __uint_as_float(v[q4 * 8 + 2 * x + 1])), il2), a0, a1);
                     w[x] = pack_bf16x2(a0, a1);
                 }
-                *reinterpret_cast<uint4 *>(srow + (cc * 4 + q4) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(srow + (c64 / 8 + q4) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
         tc_fence_before();
@@ -649,8 +669,9 @@ __global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
+        const int nw[2] = {(n_chunks + 1) / 2, n_chunks / 2};  // chunks per warpgroup
 
-        if (is_mma && lane == 0) {
+        if (ptid == 0) {
             mbar_arrive_expect_tx(kvfull, 2 * kv_tile);
             kv_armed = static_cast<int>(item_n & 1);
             const int z = b * p.T + j * p.block;
@@ -661,7 +682,7 @@ __global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
         }
         for (int i = tid; i < n_chunks * TOK; i += blockDim.x) {
             int e = -1, t = -1;
-            long long qoff = 0;
+            int qo16 = 0;
             if (i < ntok) {
                 e = p.entries[list_base + i];
                 const int qrow = e >= 0 ? e / K : -1;
@@ -671,108 +692,78 @@ __global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
                     e = -1;
                 } else {
                     t = p.T - p.n_q + (qrow - bi * p.n_q);
-                    qoff = (static_cast<long long>(qrow) * p.Hq + static_cast<long long>(hk) * G) * D;
+                    qo16 = static_cast<int>((static_cast<long long>(qrow) * p.Hq + static_cast<long long>(hk) * G) * (D / 8));
                 }
             }
             tab->entry[i] = e;
             tab->t[i] = t;
-            tab->qoff[i] = qoff;
+            tab->qo16[i] = qo16;
         }
         __syncthreads();
 
-        if (is_mma) {
-            if (lane == 0) {
-                // ---- MMA issuer: event loop over both warpgroups' chunks
-                const int nw[2] = {(n_chunks + 1) / 2, n_chunks / 2};
-                int iw[2] = {0, 0}, act[2] = {0, 0};  // act: 0 = S next, 1 = PV next
-                bool ok = mbar_wait(kvfull, item_n & 1, abort_flag, p.status);
-                kv_armed = -1;
-                const uint32_t idesc_s = idesc_bf16_f32(128, NK, false);
-                const uint32_t idesc_o = idesc_bf16_f32(128, D, true);
-                const uint32_t ka = smem_addr(kv_s), va = smem_addr(kv_s + kv_tile);
-                uint64_t t0 = global_timer_ns();
-                while (ok && (iw[0] < nw[0] || iw[1] < nw[1])) {
-                    bool progress = false;
-                    for (int x = 0; x < 2; ++x) {
-                        if (iw[x] >= nw[x]) continue;
-                        const uint32_t ts = tmem_base + static_cast<uint32_t>(x * 256);
-                        if (act[x] == 0) {
-                            if (!mbar_test(q_ready + x, mq[x] & 1)) continue;
-                            if (iw[x] > 0 && !mbar_test(bar_o + x, (mp[x] - 1) & 1)) continue;
-                            tc_fence_after();
-                            const uint32_t qa = smem_addr(q_s + (x * 2 + (iw[x] & 1)) * QBYTES);
+        if (is_prod) {
+            const int cc = ptid % PPR, r0 = ptid / PPR;
+            const uint4 *qcol = reinterpret_cast<const uint4 *>(p.q) + cc;
+            for (int c = 0; c < n_chunks; ++c) {
+                const int x = c & 1, ci = c >> 1, buf = ci & 1;
+                uint4 v[NLD];
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk)
-                                umma_bf16(ts, sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
-                                          sdesc_sw128(ka + (kk / 4) * NK * 128 + (kk % 4) * 32, 16, 1024),
-                                          idesc_s, kk > 0 ? 1u : 0u);
-                            umma_commit(bar_s + x);
-                            ++mq[x];
-                            act[x] = 1;
-                            progress = true;
-                        } else {
-                            if (!mbar_test(p_ready + x, mp[x] & 1)) continue;
-                            tc_fence_after();
-                            for (int kk = 0; kk < NK / 16; ++kk)
-                                umma_bf16_tmem_a(ts + 128, ts + kk * 8,
-                                                 sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
-                                                 idesc_o, kk > 0 ? 1u : 0u);
-                            umma_commit(bar_o + x);
-                            ++mp[x];
-                            act[x] = 0;
-                            ++iw[x];
-                            progress = true;
-                        }
-                    }
-                    if (progress) {
-                        t0 = global_timer_ns();
-                    } else if (*abort_flag) {
-                        ok = false;
-                    } else if (global_timer_ns() - t0 > kWaitLimitNs) {
-                        *abort_flag = 1;
-                        atomicOr(p.status, kDevTimeout);
-                        ok = false;
-                    }
+                for (int k = 0; k < NLD; ++k) {  // padding rows read row 0 (their output is dropped)
+                    const int r = r0 + k * RSTEP;
+                    v[k] = ld_nc_na_16(qcol + tab->qo16[c * TOK + (r >> p.log2G)] + (r & (G - 1)) * PPR);
                 }
-                if (!ok) aborted = true;
+                bool ok = true;
+                if (ci >= 2) {  // the warpgroup releases the buffer after its chunk ci - 2
+                    if (ptid == 0) ok = mbar_wait(q_free + 2 * x + buf, pf[x][buf] & 1, abort_flag, p.status);
+                    ++pf[x][buf];
+                }
+                if (named_barrier_or(kProdBar, NPROD, !ok || *abort_flag)) {
+                    aborted = true;
+                    break;
+                }
+                unsigned char *dst = q_s + (x * 2 + buf) * QBYTES + (cc / 8) * kRegionBytes;
+#pragma unroll
+                for (int k = 0; k < NLD; ++k)
+                    *reinterpret_cast<uint4 *>(dst + sw128_offset(r0 + k * RSTEP, cc % 8)) = v[k];
+                fence_proxy_async_smem();
+                named_barrier(kProdBar, NPROD);
+                if (ptid == 0) mbar_arrive(q_ready + 2 * x + buf);
             }
+            // the K/V copies have landed before the item ends (returns at once
+            // when a warpgroup already saw them; bounded otherwise)
+            if (ptid == 0 && kv_armed >= 0) mbar_drain(kvfull, static_cast<uint32_t>(kv_armed));
+            kv_armed = -1;
         } else {
             // ---- warpgroup: its chunks c = wg, wg + 2, ...
-            const int n = n_chunks > wg ? (n_chunks - wg + 1) / 2 : 0;
+            const int n = nw[wg];
             if (n > 0) {
-                gather(0, wg);
-                if (n > 1) {
-                    gather(1, wg + 2);
-                    cp_async_wait_1();
+                if (!wait_wg(kvfull, item_n & 1) || !wait_wg(q_ready + 2 * wg, qr_n[0] & 1)) {
+                    aborted = true;
                 } else {
-                    cp_async_wait_all();
+                    ++qr_n[0];
+                    if (wtid == 0) issue_s(0);
                 }
-                fence_proxy_async_smem();
-                named_barrier(wg_bar, 128);
-                if (wtid == 0) mbar_arrive(q_ready + wg);
             }
-            for (int ci = 0; ci < n; ++ci) {
+            for (int ci = 0; ci < n && !aborted; ++ci) {
                 const int c = wg + 2 * ci, buf = ci & 1;
                 if (!wait_wg(bar_s + wg, s_n & 1)) { aborted = true; break; }
                 ++s_n;
                 float m_run, l_run;
                 softmax_tile(c, m_run, l_run);
                 named_barrier(wg_bar, 128);
-                if (wtid == 0) mbar_arrive(p_ready + wg);
-                if (ci + 1 < n) {
-                    // Q of the next chunk (gathered a chunk ago) -> MMA thread
-                    cp_async_wait_all();
-                    fence_proxy_async_smem();
-                    named_barrier(wg_bar, 128);
-                    if (wtid == 0) mbar_arrive(q_ready + wg);
-                }
+                if (wtid == 0) issue_pv();
                 if (!wait_wg(bar_o + wg, o_n & 1)) { aborted = true; break; }
                 ++o_n;
+                if (ci + 1 < n) {  // S of the next chunk runs under this epilogue
+                    if (!wait_wg(q_ready + 2 * wg + (buf ^ 1), qr_n[buf ^ 1] & 1)) { aborted = true; break; }
+                    ++qr_n[buf ^ 1];
+                    if (wtid == 0) issue_s(buf ^ 1);
+                }
                 epilogue(c, m_run, l_run, q_s + (wg * 2 + buf) * QBYTES);
-                if (ci + 2 < n) {
+                if (ci + 2 < n) {  // the producers gather into this buffer again
                     bulk_wait_read_all();
                     named_barrier(wg_bar, 128);
-                    gather(buf, c + 4);
+                    if (wtid == 0) mbar_arrive(q_free + 2 * wg + buf);
                 }
             }
             bulk_wait_read_all();
@@ -784,7 +775,6 @@ __global__ void __launch_bounds__(288, 1) prefill_attn_resident_kernel(
         }
     }
     __syncthreads();
-    if (aborted && is_mma && lane == 0 && kv_armed >= 0) mbar_drain(kvfull, static_cast<uint32_t>(kv_armed));
     cp_async_wait_all();
     bulk_wait_all();
     tc_fence_before();
@@ -886,7 +876,7 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
             const int r = pc / PPR, cc = pc % PPR;
             const int ti = c * TOK + (r >> p.log2G);
             const bool ok = tab->t[ti] >= 0;
-            const __nv_bfloat16 *src = p.q + (ok ? tab->qoff[ti] + (r & (G - 1)) * D + cc * 8 : 0);
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.q) + (ok ? tab->qo16[ti] + (r & (G - 1)) * PPR + cc : 0);
             cp_async_16_ca(dst_base + (cc / 8) * kRegionBytes + sw128_offset(r, cc % 8), src,
                            ok ? 16u : 0u);
         }
@@ -1146,7 +1136,7 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
         // one division per token (tokens past the list end stay invalid)
         for (int i = tid; i < n_chunks * TOK; i += blockDim.x) {
             int e = -1, t = -1;
-            long long qoff = 0;
+            int qo16 = 0;
             if (i < ntok) {
                 e = p.entries[list_base + i];
                 const int qrow = e >= 0 ? e / K : -1;
@@ -1156,12 +1146,12 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                     e = -1;
                 } else {
                     t = p.T - p.n_q + (qrow - bi * p.n_q);
-                    qoff = (static_cast<long long>(qrow) * p.Hq + static_cast<long long>(hk) * G) * D;
+                    qo16 = static_cast<int>((static_cast<long long>(qrow) * p.Hq + static_cast<long long>(hk) * G) * (D / 8));
                 }
             }
             tab->entry[i] = e;
             tab->t[i] = t;
-            tab->qoff[i] = qoff;
+            tab->qo16[i] = qo16;
         }
         __syncthreads();
 
@@ -1324,7 +1314,7 @@ size_t prefill_attn_smem_bytes(const Shape &sh) {
     const int QBUF = NS > 1 ? 1 : 2;
     const size_t kv_tile = static_cast<size_t>(NK) * 128 * (sh.d / 64);
     const size_t q = static_cast<size_t>(sh.d / 64) * kRegionBytes + 2048;
-    return 1024 + KVST * 2 * kv_tile + 2 * QBUF * q + sizeof(ItemRows) + 128 + 32;
+    return 1024 + KVST * 2 * kv_tile + 2 * QBUF * q + sizeof(ItemRows) + 160 + 32;
 }
 
 int prefill_attn_rows_per_item(int G) {
@@ -1368,8 +1358,8 @@ cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const 
         KERNEL<<<num_sms, THREADS, smem, st>>>(tm_k, tm_v, ap);                                  \
     } while (0)
     if (ap.NS == 1) {
-        if (sh.d == 128) MSA_LAUNCH(prefill_attn_resident_kernel<128>, 288);
-        else MSA_LAUNCH(prefill_attn_resident_kernel<64>, 288);
+        if (sh.d == 128) MSA_LAUNCH(prefill_attn_resident_kernel<128>, kResidentThreads);
+        else MSA_LAUNCH(prefill_attn_resident_kernel<64>, kResidentThreads);
     } else {
         if (sh.d == 128) MSA_LAUNCH(prefill_attn_kernel<128>, 256);
         else MSA_LAUNCH(prefill_attn_kernel<64>, 256);

@@ -30,6 +30,7 @@ msa_status validate(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_idx, i
     if (static_cast<long long>(Bt) * T >= (1ll << 31)) return MSA_ERR_UNSUPPORTED;
     if (static_cast<long long>(Bt) * n_q * K >= (1ll << 31)) return MSA_ERR_UNSUPPORTED;
     if (N > kMaxBlocksPrefill) return MSA_ERR_UNSUPPORTED;
+    if (need_attn && static_cast<long long>(Bt) * n_q * Hq * d >= (1ll << 34)) return MSA_ERR_UNSUPPORTED;
     int G = 1;
     if (need_attn) {
         G = Hq / Hkv;

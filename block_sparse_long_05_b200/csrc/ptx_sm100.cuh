@@ -138,6 +138,16 @@ __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// 16-byte read-only global load that does not allocate in L1 (streams of
+// gathered rows that are used once per SM).
+__device__ __forceinline__ uint4 ld_nc_na_16(const void *src) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(src));
+    return v;
+}
+
 // ---------------------------------------------------------------- cp.async
 // 16-byte global->shared copy; src_bytes = 0 fills the destination with zeros.
 __device__ __forceinline__ void cp_async_16(void *dst, const void *src, uint32_t src_bytes) {

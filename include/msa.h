@@ -41,7 +41,8 @@
  *    weighted sum of v_i (fp32) and lse = ln sum_i exp(q.k_i / sqrt(d)).
  *  - Supported shapes: d, d_idx in {64, 128}; block in {32, 64} or a
  *    multiple of 128; 1 <= K <= 32; 128 % (Hq/Hkv) == 0; N <= 8192;
- *    Bt*T < 2^31 and Bt*n_q*K < 2^31.  Anything else
+ *    Bt*T < 2^31, Bt*n_q*K < 2^31 and Bt*n_q*Hq*d < 2^34 (the attention
+ *    calls address q in 16-byte units with 32-bit offsets).  Anything else
  *    returns MSA_ERR_UNSUPPORTED before any work is enqueued.  Tensor base
  *    pointers must be 16-byte aligned (MSA_ERR_INVALID_ARG otherwise).
  *  - Errors found on the host return immediately (nothing enqueued).  Errors a
