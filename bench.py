@@ -19,6 +19,7 @@ import json
 import os
 import statistics
 import subprocess
+import threading
 import sys
 import time
 
@@ -69,7 +70,10 @@ class ClockSampler:
         self.proc = None
         self.lines = []
 
-    def start(self):
+    def start(self, ready_timeout: float = 20.0):
+        """Start sampling; returns once the first sample has been printed, so
+        nvidia-smi's own start-up (which can stall driver calls of other
+        processes) lies before the timed region."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
@@ -77,16 +81,30 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+        first = threading.Event()
+
+        def reader():
+            for ln in self.proc.stdout:
+                self.lines.append(ln)
+                first.set()
+            first.set()
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        first.wait(ready_timeout)
 
     def stop(self):
         if not self.proc:
             return None
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+            self.proc.wait()
+        self.thread.join(timeout=5)
+        out = "".join(self.lines)
         rows = []
         for ln in out.strip().splitlines():
             parts = [p.strip() for p in ln.split(",")]

@@ -428,7 +428,7 @@ struct AttnParams {
 
 // Token table of one work item (at most kItemTokens hit-list entries),
 // built once per item in shared memory.
-constexpr int kItemTokens = 1024;
+constexpr int kItemTokens = 2048;
 struct ItemRows {
     int qo16[kItemTokens];        // offset of the token's head group hk in q, 16-byte units (0 if none)
     int entry[kItemTokens];       // list entry = partial row (b*n_q + i)*K + slot, or -1
@@ -437,31 +437,35 @@ struct ItemRows {
 
 // ===========================================================================
 // Prefill attention, K/V block resident (block <= 128): warp-specialised.
-//   warps 0-3 / 4-7: warpgroups WG0 / WG1.  Each takes alternate 128-row
-//     chunks of the item.  Per chunk: wait for S, softmax (S -> P in tensor
-//     memory), issue PV, wait for it, issue S of its next chunk (which then
-//     runs under the epilogue), epilogue (normalised bf16 partial rows staged
-//     in shared memory, one bulk copy per token).  One elected thread per
-//     warpgroup issues that warpgroup's tcgen05.mma.
-//   warps 8-11: producers.  Thread 0 of them TMA-loads K_j and V_j once per
+//   warps 0-3 / 4-7: softmax warpgroups SG0 / SG1.  Each takes alternate
+//     128-row chunks of the item: wait for S (which releases the Q tile),
+//     softmax (S -> P in tensor memory), hand the row statistics to the
+//     epilogue warpgroup, issue PV, wait for it, issue S of its next chunk.
+//     One elected thread per warpgroup issues that warpgroup's tcgen05.mma.
+//   warps 8-11: epilogue warpgroup.  For every chunk in order: read O from
+//     tensor memory (which frees it for the next PV), normalise, stage the
+//     bf16 partial rows token-major in one of two staging buffers and write
+//     each token's G rows with one bulk copy; store lse.
+//   warps 12-15: producers.  Thread 0 of them TMA-loads K_j and V_j once per
 //     item; all gather the Q rows of chunks 0, 1, 2, ... into the owning
-//     warpgroup's two Q buffers: rows are loaded into registers (not
-//     allocated in L1) before the buffer is known to be free, then stored in
+//     softmax warpgroup's Q tile: rows are loaded into registers (not
+//     allocated in L1) before the tile is known to be free, then stored in
 //     the 128-byte-swizzled layout.
-// Q readiness and Q-buffer release are mbarriers per (warpgroup, buffer), so
-// no signaller runs two phases ahead of its waiter.
-// Tensor memory: WG w owns columns [256w, 256w+256): S/P at +0, O at +128.
+// Every handshake is an mbarrier per softmax warpgroup; each side waits for
+// the other's previous phase, so no signaller runs two phases ahead.
+// Tensor memory: SG w owns columns [256w, 256w+256): S/P at +0, O at +128.
 // ===========================================================================
-constexpr int kResidentThreads = 384;
+constexpr int kResidentThreads = 512;
 
 template <int D>
 __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     AttnParams p) {
     constexpr int DREG = D / 64;
-    constexpr uint32_t QBYTES = DREG * kRegionBytes + 2048;  // Q tile + staging room
+    constexpr uint32_t QT = DREG * kRegionBytes;   // Q tile
+    constexpr uint32_t STB = QT + 2048;            // staging: 16-byte pad per token
     constexpr int PPR = D / 8;        // 16-byte pieces per row
-    constexpr int NPROD = 128;        // producer threads (warps 8-11)
+    constexpr int NPROD = 128;        // producer threads (warps 12-15)
     constexpr int NLD = PPR;          // pieces per producer thread per chunk
     constexpr int RSTEP = NPROD / PPR;
     const int NK = p.NK;
@@ -470,32 +474,34 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = align1024(smem_raw);
     unsigned char *kv_s = base;                        // K tile, V tile
-    unsigned char *q_s = kv_s + 2 * kv_tile;           // [wg][buf]
-    ItemRows *tab = reinterpret_cast<ItemRows *>(q_s + 4 * QBYTES);
+    unsigned char *q_s = kv_s + 2 * kv_tile;           // Q tile [sg]
+    unsigned char *st_s = q_s + 2 * QT;                // staging [2]
+    float2 *ml_s = reinterpret_cast<float2 *>(st_s + 2 * STB);  // (m, l) [sg][row]
+    ItemRows *tab = reinterpret_cast<ItemRows *>(ml_s + 2 * 128);
     uint64_t *kvfull = reinterpret_cast<uint64_t *>(tab + 1);
-    uint64_t *bar_s = kvfull + 1;     // [wg]      S(w, i) complete
-    uint64_t *bar_o = kvfull + 3;     // [wg]      PV(w, i) complete
-    uint64_t *q_ready = kvfull + 5;   // [wg][buf] Q tile gathered
-    uint64_t *q_free = kvfull + 9;    // [wg][buf] Q buffer released by its warpgroup
+    uint64_t *bar_s = kvfull + 1;      // [sg] S complete
+    uint64_t *bar_o = kvfull + 3;      // [sg] PV complete
+    uint64_t *q_ready = kvfull + 5;    // [sg] Q tile gathered
+    uint64_t *q_free = kvfull + 7;     // [sg] Q tile read by S
+    uint64_t *ml_ready = kvfull + 9;   // [sg] row statistics written
+    uint64_t *o_free = kvfull + 11;    // [sg] O read by the epilogue warpgroup
     int *sh_item = reinterpret_cast<int *>(kvfull + 13);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sh_item + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid / 32;
-    const bool is_prod = warp >= 8;
-    const int ptid = tid - 256;  // producer thread index
-    const int wg = is_prod ? 0 : (warp >> 2), wtid = tid & 127;
-    const uint32_t wg_bar = 1 + wg;
-    constexpr uint32_t kProdBar = 3;
+    const int role = warp >> 2;        // 0, 1: softmax; 2: epilogue; 3: producers
+    const int wg = role & 1, wtid = tid & 127;
+    const uint32_t role_bar = 1 + role;
     if (tid == 0) {
         mbar_init(kvfull, 1);
         for (int w = 0; w < 2; ++w) {
             mbar_init(bar_s + w, 1);
             mbar_init(bar_o + w, 1);
-            for (int u = 0; u < 2; ++u) {
-                mbar_init(q_ready + 2 * w + u, 1);
-                mbar_init(q_free + 2 * w + u, 1);
-            }
+            mbar_init(q_ready + w, 1);
+            mbar_init(q_free + w, 1);
+            mbar_init(ml_ready + w, 1);
+            mbar_init(o_free + w, 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -513,6 +519,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     const uint32_t tmem_s = tmem_base + static_cast<uint32_t>(wg * 256);
     const uint32_t tmem_o = tmem_s + 128;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint64_t pol_first = l2_policy_evict_first(), pol_last = l2_policy_evict_last();
 
     const int n_items = p.counters[0];
     const int total = n_items * p.Hkv;
@@ -520,24 +527,26 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     const int row = wtid;
     const int tok = row >> p.log2G, g = row & (G - 1);
 
-    uint32_t s_n = 0, o_n = 0, item_n = 0;   // warpgroup: bar_s / bar_o phases
-    uint32_t qr_n[2] = {0, 0};                // warpgroup: q_ready phases per buffer
-    uint32_t pf[2][2] = {{0, 0}, {0, 0}};     // producers: q_free phases
+    // phase counters (each thread keeps those of its own role)
+    uint32_t s_n = 0, pv_n = 0, qr_n = 0, item_n = 0;  // softmax warpgroup
+    uint32_t eo_n[2] = {0, 0}, ec_n = 0;                // epilogue: per-sg chunks, all chunks
+    uint32_t pf[2] = {0, 0};                            // producers: q_free phases
     int kv_armed = -1;
     bool aborted = false;
     int cur_j = 0, cur_hk = 0;
 
-    auto wait_wg = [&](uint64_t *bar, uint32_t parity) -> bool {
+    // bounded wait of the role's thread 0, outcome shared by the role's 128 threads
+    auto wait_role = [&](uint64_t *bar, uint32_t parity) -> bool {
         bool ok = true;
         if (wtid == 0) ok = mbar_wait(bar, parity, abort_flag, p.status);
-        return !named_barrier_or(wg_bar, 128, !ok || *abort_flag);
+        return !named_barrier_or(role_bar, 128, !ok || *abort_flag);
     };
     const uint32_t idesc_s = idesc_bf16_f32(128, NK, false);
     const uint32_t idesc_o = idesc_bf16_f32(128, D, true);
-    // S = Q K^T for the Q tile in buffer `buf` (elected thread)
-    auto issue_s = [&](int buf) {
+    // S = Q K^T for the warpgroup's Q tile (elected thread)
+    auto issue_s = [&]() {
         tc_fence_after();
-        const uint32_t qa = smem_addr(q_s + (wg * 2 + buf) * QBYTES), ka = smem_addr(kv_s);
+        const uint32_t qa = smem_addr(q_s + wg * QT), ka = smem_addr(kv_s);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
             umma_bf16(tmem_s, sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
@@ -613,32 +622,49 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         tc_fence_before();
     };
 
-    // normalised bf16 partial rows staged token-major (16-byte pad per token)
-    // in `stage`, one bulk copy per token; lse stored directly
-    auto epilogue = [&](int c, float m_run, float l_run, unsigned char *stage) {
+    // epilogue warpgroup, chunk c of softmax warpgroup w: normalised bf16
+    // partial rows of O staged token-major (16-byte pad per token), one bulk
+    // copy per token; lse stored directly.  Returns false on abort.
+    auto epilogue = [&](int c, int w) -> bool {
+        if (!wait_role(bar_o + w, eo_n[w] & 1) || !wait_role(ml_ready + w, eo_n[w] & 1)) return false;
+        ++eo_n[w];
+        const float2 ml = ml_s[w * 128 + row];
+        const float m_run = ml.x, l_run = ml.y;
+        unsigned char *stage = st_s + (ec_n & 1) * STB;
+        ++ec_n;
+        // the bulk copies that last read this staging buffer (two chunks ago) are done
+        if (g == 0) bulk_wait_read_1();
+        if (G <= 32)
+            __syncwarp();
+        else
+            named_barrier(role_bar, 128);
         tc_fence_after();
+        const uint32_t to = tmem_base + static_cast<uint32_t>(w * 256 + 128);
         const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
         const uint64_t il2 = f2_pack(inv_l, inv_l);
         const uint32_t tok_bytes = static_cast<uint32_t>(G * D * 2 + 16);
         unsigned char *srow = stage + tok * tok_bytes + g * (D * 2);
 #pragma unroll
-        for (int c64 = 0; c64 < D; c64 += 32) {
+        for (int c32 = 0; c32 < D; c32 += 32) {
             uint32_t v[32];
-            tmem_ld32(tmem_o + lane_addr + c64, v);
+            tmem_ld32(to + lane_addr + c32, v);
             tmem_wait_ld();
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t w[4];
+                uint32_t wv[4];
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
                     float a0, a1;
                     f2_unpack(f2_mul(f2_pack(__uint_as_float(v[q4 * 8 + 2 * x]), __uint_as_float(v[q4 * 8 + 2 * x + 1])), il2), a0, a1);
-                    w[x] = pack_bf16x2(a0, a1);
+                    wv[x] = pack_bf16x2(a0, a1);
                 }
-                *reinterpret_cast<uint4 *>(srow + (c64 / 8 + q4) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(srow + (c32 / 8 + q4) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
         }
+        // O and the row statistics have been read: the warpgroup may issue its next PV
         tc_fence_before();
+        named_barrier(role_bar, 128);
+        if (wtid == 0) mbar_arrive(o_free + w);
         const int e = tab->entry[c * TOK + tok];
         if (e >= 0) {
             const long long prow = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G + g;
@@ -648,12 +674,15 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         if (G <= 32)
             __syncwarp();
         else
-            named_barrier(wg_bar, 128);
-        if (g == 0 && e >= 0) {
-            const long long prow0 = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G;
-            bulk_store(p.part_o + prow0 * D, stage + tok * tok_bytes, static_cast<uint32_t>(G * D * 2));
-            bulk_commit();
+            named_barrier(role_bar, 128);
+        if (g == 0) {
+            if (e >= 0) {
+                const long long prow0 = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G;
+                bulk_store_hint(p.part_o + prow0 * D, stage + tok * tok_bytes, static_cast<uint32_t>(G * D * 2), pol_first);
+            }
+            bulk_commit();  // one group per chunk (possibly empty) keeps the count in step
         }
+        return true;
     };
 
     while (true) {
@@ -669,9 +698,8 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
-        const int nw[2] = {(n_chunks + 1) / 2, n_chunks / 2};  // chunks per warpgroup
 
-        if (ptid == 0) {
+        if (role == 3 && wtid == 0) {
             mbar_arrive_expect_tx(kvfull, 2 * kv_tile);
             kv_armed = static_cast<int>(item_n & 1);
             const int z = b * p.T + j * p.block;
@@ -701,72 +729,80 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         }
         __syncthreads();
 
-        if (is_prod) {
-            const int cc = ptid % PPR, r0 = ptid / PPR;
+        if (role == 3) {
+            // ---- producers
+            const int cc = wtid % PPR, r0 = wtid / PPR;
             const uint4 *qcol = reinterpret_cast<const uint4 *>(p.q) + cc;
             for (int c = 0; c < n_chunks; ++c) {
-                const int x = c & 1, ci = c >> 1, buf = ci & 1;
+                const int x = c & 1, ci = c >> 1;
                 uint4 v[NLD];
 #pragma unroll
                 for (int k = 0; k < NLD; ++k) {  // padding rows read row 0 (their output is dropped)
                     const int r = r0 + k * RSTEP;
-                    v[k] = ld_nc_na_16(qcol + tab->qo16[c * TOK + (r >> p.log2G)] + (r & (G - 1)) * PPR);
+                    v[k] = ld_nc_na_16_hint(qcol + tab->qo16[c * TOK + (r >> p.log2G)] + (r & (G - 1)) * PPR, pol_last);
                 }
-                bool ok = true;
-                if (ci >= 2) {  // the warpgroup releases the buffer after its chunk ci - 2
-                    if (ptid == 0) ok = mbar_wait(q_free + 2 * x + buf, pf[x][buf] & 1, abort_flag, p.status);
-                    ++pf[x][buf];
+                if (ci >= 1) {  // S of the warpgroup's chunk ci - 1 has read the tile
+                    if (!wait_role(q_free + x, pf[x] & 1)) {
+                        aborted = true;
+                        break;
+                    }
+                    ++pf[x];
                 }
-                if (named_barrier_or(kProdBar, NPROD, !ok || *abort_flag)) {
-                    aborted = true;
-                    break;
-                }
-                unsigned char *dst = q_s + (x * 2 + buf) * QBYTES + (cc / 8) * kRegionBytes;
+                unsigned char *dst = q_s + x * QT + (cc / 8) * kRegionBytes;
 #pragma unroll
                 for (int k = 0; k < NLD; ++k)
                     *reinterpret_cast<uint4 *>(dst + sw128_offset(r0 + k * RSTEP, cc % 8)) = v[k];
                 fence_proxy_async_smem();
-                named_barrier(kProdBar, NPROD);
-                if (ptid == 0) mbar_arrive(q_ready + 2 * x + buf);
+                named_barrier(role_bar, 128);
+                if (wtid == 0) mbar_arrive(q_ready + x);
             }
             // the K/V copies have landed before the item ends (returns at once
             // when a warpgroup already saw them; bounded otherwise)
-            if (ptid == 0 && kv_armed >= 0) mbar_drain(kvfull, static_cast<uint32_t>(kv_armed));
+            if (wtid == 0 && kv_armed >= 0) mbar_drain(kvfull, static_cast<uint32_t>(kv_armed));
             kv_armed = -1;
+        } else if (role == 2) {
+            // ---- epilogue warpgroup: every chunk of the item in order
+            for (int c = 0; c < n_chunks; ++c)
+                if (!epilogue(c, c & 1)) {
+                    aborted = true;
+                    break;
+                }
         } else {
-            // ---- warpgroup: its chunks c = wg, wg + 2, ...
-            const int n = nw[wg];
+            // ---- softmax warpgroup: its chunks c = wg, wg + 2, ...
+            const int n = (n_chunks + 1 - wg) / 2;
             if (n > 0) {
-                if (!wait_wg(kvfull, item_n & 1) || !wait_wg(q_ready + 2 * wg, qr_n[0] & 1)) {
+                if (!wait_role(kvfull, item_n & 1) || !wait_role(q_ready + wg, qr_n & 1)) {
                     aborted = true;
                 } else {
-                    ++qr_n[0];
-                    if (wtid == 0) issue_s(0);
+                    ++qr_n;
+                    if (wtid == 0) issue_s();
                 }
             }
             for (int ci = 0; ci < n && !aborted; ++ci) {
-                const int c = wg + 2 * ci, buf = ci & 1;
-                if (!wait_wg(bar_s + wg, s_n & 1)) { aborted = true; break; }
+                const int c = wg + 2 * ci;
+                if (!wait_role(bar_s + wg, s_n & 1)) { aborted = true; break; }
                 ++s_n;
+                if (wtid == 0 && ci + 1 < n) mbar_arrive(q_free + wg);
                 float m_run, l_run;
                 softmax_tile(c, m_run, l_run);
-                named_barrier(wg_bar, 128);
-                if (wtid == 0) issue_pv();
-                if (!wait_wg(bar_o + wg, o_n & 1)) { aborted = true; break; }
-                ++o_n;
-                if (ci + 1 < n) {  // S of the next chunk runs under this epilogue
-                    if (!wait_wg(q_ready + 2 * wg + (buf ^ 1), qr_n[buf ^ 1] & 1)) { aborted = true; break; }
-                    ++qr_n[buf ^ 1];
-                    if (wtid == 0) issue_s(buf ^ 1);
+                // the epilogue warpgroup has read O and (m, l) of the previous PV
+                if (pv_n > 0 && !wait_role(o_free + wg, (pv_n - 1) & 1)) { aborted = true; break; }
+                ml_s[wg * 128 + row] = make_float2(m_run, l_run);
+                named_barrier(role_bar, 128);
+                if (wtid == 0) {
+                    mbar_arrive(ml_ready + wg);
+                    issue_pv();
                 }
-                epilogue(c, m_run, l_run, q_s + (wg * 2 + buf) * QBYTES);
-                if (ci + 2 < n) {  // the producers gather into this buffer again
-                    bulk_wait_read_all();
-                    named_barrier(wg_bar, 128);
-                    if (wtid == 0) mbar_arrive(q_free + 2 * wg + buf);
+                ++pv_n;
+                if (ci + 1 < n) {  // S of the next chunk once PV has read P
+                    if (!wait_role(bar_o + wg, (pv_n - 1) & 1) || !wait_role(q_ready + wg, qr_n & 1)) {
+                        aborted = true;
+                        break;
+                    }
+                    ++qr_n;
+                    if (wtid == 0) issue_s();
                 }
             }
-            bulk_wait_read_all();
         }
         ++item_n;
         if (__syncthreads_or(aborted)) {
@@ -775,7 +811,6 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         }
     }
     __syncthreads();
-    cp_async_wait_all();
     bulk_wait_all();
     tc_fence_before();
     __syncthreads();
@@ -1314,12 +1349,14 @@ size_t prefill_attn_smem_bytes(const Shape &sh) {
     const int QBUF = NS > 1 ? 1 : 2;
     const size_t kv_tile = static_cast<size_t>(NK) * 128 * (sh.d / 64);
     const size_t q = static_cast<size_t>(sh.d / 64) * kRegionBytes + 2048;
+    if (NS == 1)  // resident kernel: K/V, two Q tiles, two staging buffers, row statistics
+        return 1024 + 2 * kv_tile + 2 * (q - 2048) + 2 * q + 2 * 128 * 8 + sizeof(ItemRows) + 160 + 32;
     return 1024 + KVST * 2 * kv_tile + 2 * QBUF * q + sizeof(ItemRows) + 160 + 32;
 }
 
 int prefill_attn_rows_per_item(int G) {
     const int tok = 128 / G;
-    return 16 * tok < kItemTokens ? 16 * tok : kItemTokens;
+    return 32 * tok < kItemTokens ? 32 * tok : kItemTokens;
 }
 
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,

@@ -85,6 +85,8 @@ def test_sparse_attn_host_validation(lib):
     assert call(*ok, 1, 8, 8, 8, 2, 64, 64, 4, FAKE, 64, None) == 3        # ws small
     # prefill with more than 8192 blocks is outside the supported shapes
     assert call(*ok, 1, 2, 8193 * 32, 8, 2, 64, 32, 4, FAKE, 1 << 40, None) == 2
+    # q larger than 2^34 elements (offsets are 32-bit in 16-byte units)
+    assert call(*ok, 1, 1 << 20, 1 << 20, 128, 1, 128, 128, 4, FAKE, 1 << 50, None) == 2
 
 
 def test_select_invert_host_validation(lib):
