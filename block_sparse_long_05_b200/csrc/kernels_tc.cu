@@ -565,47 +565,68 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         umma_commit(bar_o + wg);
     };
 
-    // softmax of this thread's row in two passes over tensor memory: row max,
-    // then P = 2^(s*c - m) as bf16 written over the columns of S already read
+    // Softmax of this thread's row in one pass over tensor memory, 32 columns
+    // at a time.  P = 2^(s*c - m_ref) with m_ref the first group's maximum;
+    // a later group whose maximum exceeds m_ref by more than 8 (log2 units)
+    // raises m_ref and rescales the P columns already written and the sum
+    // (rare; any m_ref gives the same O / l and lse, it only has to keep the
+    // terms in range).  P is written as bf16 over the S columns already read.
+    // Rows away from the diagonal block skip the causal mask (warp-uniform).
     auto softmax_tile = [&](int c, float &m_run, float &l_run) {
         tc_fence_after();
         const int t = tab->t[c * TOK + tok];
         const int lim = t - cur_j * p.block;  // valid key columns: <= lim
-        const bool masked = lim < NK - 1;
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const bool wmask = __any_sync(0xffffffffu, lim < NK - 1);
+        const float sc = p.scale_log2;
+        const uint64_t sc2 = f2_pack(sc, sc);
+        float mref = -INFINITY;
+        float lsum = 0.f;
         for (int cc = 0; cc < NK / 32; ++cc) {
             uint32_t v[32];
             tmem_ld32(tmem_s + lane_addr + cc * 32, v);
             tmem_wait_ld();
-            float sv[32];
+            if (wmask) {
 #pragma unroll
-            for (int x = 0; x < 32; ++x)
-                sv[x] = (masked && cc * 32 + x > lim) ? -INFINITY : __uint_as_float(v[x]);
-#pragma unroll
-            for (int x = 0; x < 32; x += 8) {
-                m4[0] = fmax3(m4[0], sv[x], sv[x + 1]);
-                m4[1] = fmax3(m4[1], sv[x + 2], sv[x + 3]);
-                m4[2] = fmax3(m4[2], sv[x + 4], sv[x + 5]);
-                m4[3] = fmax3(m4[3], sv[x + 6], sv[x + 7]);
+                for (int x = 0; x < 32; ++x)
+                    if (cc * 32 + x > lim) v[x] = __float_as_uint(-INFINITY);
             }
-        }
-        m_run = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * p.scale_log2;
-        const float mref = m_run == -INFINITY ? 0.f : m_run;
-        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2_pack(-mref, -mref);
-        uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
-        for (int cc = 0; cc < NK / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tmem_s + lane_addr + cc * 32, v);
-            tmem_wait_ld();
+            float g4[4] = {__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]), __uint_as_float(v[3])};
+#pragma unroll
+            for (int x = 4; x < 32; x += 8) {
+                g4[0] = fmax3(g4[0], __uint_as_float(v[x]), __uint_as_float(v[x + 4]));
+                g4[1] = fmax3(g4[1], __uint_as_float(v[x + 1]), __uint_as_float(v[x + 5]));
+                g4[2] = fmax3(g4[2], __uint_as_float(v[x + 2]), __uint_as_float(v[x + 6]));
+                g4[3] = fmax3(g4[3], __uint_as_float(v[x + 3]), __uint_as_float(v[x + 7]));
+            }
+            const float gm = fmaxf(fmax3(g4[0], g4[1], g4[2]), g4[3]) * sc;
+            if (__any_sync(0xffffffffu, gm > mref + 8.f)) {
+                const float mnew = fmaxf(mref, gm);
+                // factor for what was accumulated with the old reference
+                const float f = (mref == -INFINITY || mnew == -INFINITY) ? 0.f : ex2_approx(mref - mnew);
+                if (cc > 0) tmem_wait_st();  // the P groups written so far are readable
+                for (int g = 0; g < cc; ++g) {  // warp-collective; f = 1 leaves a row unchanged
+                    uint32_t w16[16];
+                    tmem_ld16(tmem_s + lane_addr + g * 16, w16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w16[x]);
+                        w16[x] = pack_bf16x2(__low2float(h) * f, __high2float(h) * f);
+                    }
+                    tmem_st16(tmem_s + lane_addr + g * 16, w16);
+                }
+                lsum *= f;
+                mref = mnew;
+            }
+            const float mr = mref == -INFINITY ? 0.f : mref;
+            const uint64_t nm2 = f2_pack(-mr, -mr);
+            uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
             uint32_t w16[16];
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
-                const float s0 = (masked && cc * 32 + 2 * x > lim) ? -INFINITY : __uint_as_float(v[2 * x]);
-                const float s1 = (masked && cc * 32 + 2 * x + 1 > lim) ? -INFINITY : __uint_as_float(v[2 * x + 1]);
                 float a0, a1;
-                f2_unpack(f2_fma(f2_pack(s0, s1), sc2, nm2), a0, a1);
-                const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * x]), __uint_as_float(v[2 * x + 1])), sc2, nm2), a0, a1);
+                const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);  // masked (-inf) columns give 0
                 if (x & 1)
                     ls2b = f2_add(ls2b, f2_pack(p0, p1));
                 else
@@ -613,11 +634,13 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
                 w16[x] = pack_bf16x2(p0, p1);
             }
             tmem_st16(tmem_s + lane_addr + cc * 16, w16);
+            float la0, la1, lb0, lb1;
+            f2_unpack(ls2a, la0, la1);
+            f2_unpack(ls2b, lb0, lb1);
+            lsum += (la0 + la1) + (lb0 + lb1);
         }
-        float la0, la1, lb0, lb1;
-        f2_unpack(ls2a, la0, la1);
-        f2_unpack(ls2b, lb0, lb1);
-        l_run = (la0 + la1) + (lb0 + lb1);
+        m_run = mref;
+        l_run = lsum;
         tmem_wait_st();
         tc_fence_before();
     };

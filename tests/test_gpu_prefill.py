@@ -125,6 +125,24 @@ def test_attention_random_selection(w):
     _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)
 
 
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[2], SMALL[3]], ids=lambda w: w.name)
+@pytest.mark.parametrize("rising", [True, False], ids=["rising", "falling"])
+def test_attention_score_spread(w, rising):
+    # Keys far apart in score within one block (x6 on one side of the block),
+    # so a row's largest scores sit in a later (rising) or the first (falling)
+    # 32-key group: exercises the softmax reference-max updates.
+    lib_ready()
+    x = make_inputs(w, device="cuda")
+    pos = torch.arange(w.T, device="cuda") % w.block
+    big = (pos >= w.block // 2) if rising else (pos < 32)
+    scale = torch.where(big, 6.0, 1.0).to(torch.float32)
+    x["k"] = (x["k"].float() * scale.view(1, -1, 1, 1)).to(torch.bfloat16)
+    ids = random_selection(w, device="cuda")
+    out, lse = run_attn(w, x, ids, _ws(w))
+    rows = torch.arange(w.Bt * w.n_q, dtype=torch.int64)
+    _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)
+
+
 @pytest.mark.parametrize("w", [PREFILL_64K, PREFILL_256K], ids=lambda w: w.name)
 def test_prefill_full_size_sampled(w):
     _end_to_end(w, rows=sample_rows(w, N_SAMPLE))
