@@ -294,7 +294,7 @@ def run_msa(args, rank, world, local_rank):
     bound, work = cands[dom]
     kern_ms = sm[dom]
     kernel_names = {"index0": "prefill_index_kernel" if not w.is_decode else "decode_index_scan_kernel",
-                    "attn1": ("prefill_attn_resident_kernel" if w.block <= 128 else "prefill_attn_kernel")
+                    "attn1": ("prefill_attn_resident_kernel" if w.block <= 128 else "prefill_attn_streamed_kernel")
                     if not w.is_decode else "decode_attn_kernel"}
     if bound == "tensor":
         achieved = work / (kern_ms / 1e3) / 1e12

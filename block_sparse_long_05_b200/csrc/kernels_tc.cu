@@ -668,12 +668,13 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         const uint32_t tok_bytes = static_cast<uint32_t>(G * D * 2 + 16);
         unsigned char *srow = stage + tok * tok_bytes + g * (D * 2);
 #pragma unroll
-        for (int c32 = 0; c32 < D; c32 += 32) {
-            uint32_t v[32];
-            tmem_ld32(to + lane_addr + c32, v);
+        for (int c64 = 0; c64 < D; c64 += 64) {
+            uint32_t v[64];
+            tmem_ld32(to + lane_addr + c64, *reinterpret_cast<uint32_t(*)[32]>(v));
+            tmem_ld32(to + lane_addr + c64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
             tmem_wait_ld();
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q4 = 0; q4 < 8; ++q4) {
                 uint32_t wv[4];
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
@@ -681,7 +682,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
                     f2_unpack(f2_mul(f2_pack(__uint_as_float(v[q4 * 8 + 2 * x]), __uint_as_float(v[q4 * 8 + 2 * x + 1])), il2), a0, a1);
                     wv[x] = pack_bf16x2(a0, a1);
                 }
-                *reinterpret_cast<uint4 *>(srow + (c32 / 8 + q4) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                *reinterpret_cast<uint4 *>(srow + (c64 / 8 + q4) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
         }
         // O and the row statistics have been read: the warpgroup may issue its next PV
@@ -840,44 +841,87 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     if (warp == 0) tmem_dealloc(tmem_base, 512);
 }
 
+// ===========================================================================
+// Prefill attention, K/V block streamed (block > 128): warp-specialised.
+// A block of NS * 128 keys is streamed as NS sub-tiles; each chunk of 128
+// tile rows sees all of them in order, with O accumulated in tensor memory.
+//   warps 0-3 / 4-7: softmax warpgroups SG0 / SG1, alternate chunks (SG0
+//     takes chunk 2r, SG1 chunk 2r + 1 of round r).  Per sub-tile: wait for
+//     S, softmax against the chunk's running reference maximum (a rise by
+//     more than 8 rescales the P columns written so far, the running sum
+//     and, past the first sub-tile, O), hand P to the MMA thread; after the
+//     last sub-tile hand (m, l) to the epilogue warpgroup.
+//   warps 8-11: epilogue warpgroup, as in the resident kernel (one staging
+//     buffer).
+//   warp 12 (one thread): streams K and V sub-tiles through a ring of three
+//     tile slots (TMA) and issues every tcgen05.mma: S(x, r, s) once K_s and
+//     (for s = 0) Q of the chunk are in, and PV(x, r, s - 1) has completed;
+//     PV(x, r, s) once P is in tensor memory and V_s is in.  A slot is
+//     refilled when every reader of its tile has completed (commit).
+//   warps 13-15: producers, gathering each chunk's Q rows (two halves per
+//     tile, registers, evict-last) into the owning warpgroup's Q tile.
+// Tensor memory: SG w owns columns [256w, 256w+256): S/P at +0, O at +128.
+// ===========================================================================
+constexpr int kStreamedThreads = 512;
+constexpr int kKvSlots = 3;
+
 template <int D>
-__global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
+__global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     AttnParams p) {
-    constexpr int DREG = D / 64;                 // swizzled regions per Q row block
-    // Q tile (DREG swizzled regions) plus room for the epilogue's staging
-    // layout, which pads every token by 16 bytes (at most 128 tokens)
-    constexpr uint32_t QBYTES = DREG * kRegionBytes + 2048;
-    constexpr int PPR = D / 8;                   // 16-byte pieces per Q row
-    const int NK = p.NK;
-    const uint32_t kv_tile = static_cast<uint32_t>(NK) * 128u * DREG;  // one of K or V
-    const bool streamed = p.NS > 1;
-    const int KVST = streamed ? 2 : 1;
-    const int QBUF = streamed ? 1 : 2;
+    constexpr int DREG = D / 64;
+    constexpr uint32_t QT = DREG * kRegionBytes;   // Q tile
+    constexpr uint32_t STB = QT + 2048;            // staging: 16-byte pad per token
+    constexpr int PPR = D / 8;                     // 16-byte pieces per row
+    constexpr int NPROD = 96;                      // producer threads (warps 13-15)
+    constexpr int RSTEP = NPROD / PPR;             // rows between a thread's pieces
+    constexpr int NLDH = (64 + RSTEP - 1) / RSTEP; // pieces per thread per half tile
+    const int NK = p.NK, NS = p.NS;
+    const uint32_t kv_tile = static_cast<uint32_t>(NK) * 128u * DREG;  // one K or V sub-tile
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = align1024(smem_raw);
-    unsigned char *kv_s = base;                                   // KVST x (K tile, V tile)
-    unsigned char *q_s = kv_s + KVST * 2 * kv_tile;               // [wg][buf] Q tiles
-    unsigned char *tail = q_s + 2 * QBUF * QBYTES;
-    ItemRows *tab = reinterpret_cast<ItemRows *>(tail);
-    uint64_t *kvfull = reinterpret_cast<uint64_t *>(tab + 1);     // [2]
-    uint64_t *bar_s = kvfull + 2;                                 // [wg]
-    uint64_t *bar_o = kvfull + 4;                                 // [wg]
-    int *sh_item = reinterpret_cast<int *>(kvfull + 6);
+    unsigned char *kv_s = base;                             // kKvSlots tile slots
+    unsigned char *q_s = kv_s + kKvSlots * kv_tile;         // Q tile [sg]
+    unsigned char *st_s = q_s + 2 * QT;                     // staging
+    float2 *ml_s = reinterpret_cast<float2 *>(st_s + STB);  // (m, l) [sg][row]
+    ItemRows *tab = reinterpret_cast<ItemRows *>(ml_s + 2 * 128);
+    uint64_t *kvfull = reinterpret_cast<uint64_t *>(tab + 1);  // [slot] tile landed
+    uint64_t *slot_free = kvfull + 3;  // [slot] every reader of the slot's tile completed
+    uint64_t *bar_s = kvfull + 6;      // [sg] S complete
+    uint64_t *bar_pv = kvfull + 8;     // [sg] a PV complete
+    uint64_t *bar_o = kvfull + 10;     // [sg] last PV of a chunk complete
+    uint64_t *q_ready = kvfull + 12;   // [sg] Q tile gathered
+    uint64_t *q_free = kvfull + 14;    // [sg] Q tile read by the chunk's last S
+    uint64_t *ml_ready = kvfull + 16;  // [sg] row statistics written
+    uint64_t *o_free = kvfull + 18;    // [sg] O read by the epilogue warpgroup
+    uint64_t *p_ready = kvfull + 20;   // [sg] P in tensor memory
+    int *sh_item = reinterpret_cast<int *>(kvfull + 22);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sh_item + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
-    const int tid = threadIdx.x, warp = tid / 32;
-    const int wg = tid >> 7, wtid = tid & 127;
-    const uint32_t wg_bar = 1 + wg;  // named barrier per warpgroup
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid & 31;
+    // 0, 1: softmax; 2: epilogue; 3: MMA / K-V thread; 4: producers
+    const int role = warp < 12 ? (warp >> 2) : (warp == 12 ? 3 : 4);
+    const int wg = role & 1, wtid = tid & 127;
+    const int ptid = tid - 13 * 32;    // producer thread index
+    const uint32_t role_bar = 1 + role;
+    const uint32_t role_threads = role == 4 ? NPROD : 128;
     if (tid == 0) {
-        mbar_init(kvfull, 1);
-        mbar_init(kvfull + 1, 1);
-        mbar_init(bar_s, 1);
-        mbar_init(bar_s + 1, 1);
-        mbar_init(bar_o, 1);
-        mbar_init(bar_o + 1, 1);
+        for (int sl = 0; sl < kKvSlots; ++sl) {
+            mbar_init(kvfull + sl, 1);
+            mbar_init(slot_free + sl, 1);
+        }
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(bar_s + w, 1);
+            mbar_init(bar_pv + w, 1);
+            mbar_init(bar_o + w, 1);
+            mbar_init(q_ready + w, 1);
+            mbar_init(q_free + w, 1);
+            mbar_init(ml_ready + w, 1);
+            mbar_init(o_free + w, 1);
+            mbar_init(p_ready + w, 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_k);
@@ -890,161 +934,94 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot + static_cast<uint32_t>(wg * 256);
-    const uint32_t tmem_s = tmem;        // S (fp32) / P (bf16 pairs)
-    const uint32_t tmem_o = tmem + 128;  // O (fp32)
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_s = tmem_base + static_cast<uint32_t>(wg * 256);
+    const uint32_t tmem_o = tmem_s + 128;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint64_t pol_first = l2_policy_evict_first(), pol_last = l2_policy_evict_last();
 
     const int n_items = p.counters[0];
     const int total = n_items * p.Hkv;
     const int G = p.G, TOK = p.TOK, K = p.K;
-    const uint32_t idesc_s = idesc_bf16_f32(128, NK, false);
-    const uint32_t idesc_o = idesc_bf16_f32(128, D, true);
-    const int row = wtid;                // M row = TMEM lane of this thread
+    const int row = wtid;
     const int tok = row >> p.log2G, g = row & (G - 1);
 
-    uint32_t kv_issue = 0, kv_use = 0, s_n = 0, o_n = 0, item_n = 0;
-    int armed_parity[2] = {-1, -1};
+    // phase counters (each thread keeps those of its own role)
+    uint32_t s_n = 0, pv_n = 0, och = 0, item_n = 0;  // softmax warpgroup
+    uint32_t eo_n[2] = {0, 0};                         // epilogue
+    uint32_t mq[2] = {0, 0}, mp[2] = {0, 0}, gt = 0;   // MMA thread: S rounds, PVs, tiles loaded
+    uint32_t pf[2] = {0, 0};                           // producers
     bool aborted = false;
-    int cur_b = 0, cur_j = 0, cur_hk = 0;
+    int cur_j = 0, cur_hk = 0;
 
-    // K/V loads of sub-tile kt of block (b, j), kv head hk (thread 0 only).
-    auto issue_kv = [&](int b, int j, int hk, int kt) {
-        const uint32_t st = kv_issue % KVST;
-        unsigned char *kd = kv_s + st * 2 * kv_tile;
-        unsigned char *vd = kd + kv_tile;
-        mbar_arrive_expect_tx(kvfull + st, 2 * kv_tile);
-        armed_parity[st] = static_cast<int>((kv_issue / KVST) & 1);
-        const int z = b * p.T + j * p.block + kt * NK;
-        for (int r = 0; r < DREG; ++r) {
-            tma_load_3d(kd + r * NK * 128, &tm_k, kvfull + st, r * 64, hk, z);
-            tma_load_3d(vd + r * NK * 128, &tm_v, kvfull + st, r * 64, hk, z);
-        }
-        ++kv_issue;
-    };
-
-    // cp.async gather of the 128 Q rows of chunk `c` (row = tk*G + g) into
-    // q_s[wg][buf].  Piece pc = wtid + 128*k is 16-byte chunk pc % PPR of row
-    // pc / PPR, so one warp instruction covers whole 2*D-byte rows (coalesced).
-    // Called by one whole warpgroup.
-    auto gather = [&](int buf, int c) {
-        unsigned char *dst_base = q_s + (wg * QBUF + buf) * QBYTES;
-#pragma unroll 4
-        for (int pc = wtid; pc < 128 * PPR; pc += 128) {
-            const int r = pc / PPR, cc = pc % PPR;
-            const int ti = c * TOK + (r >> p.log2G);
-            const bool ok = tab->t[ti] >= 0;
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.q) + (ok ? tab->qo16[ti] + (r & (G - 1)) * PPR + cc : 0);
-            cp_async_16_ca(dst_base + (cc / 8) * kRegionBytes + sw128_offset(r, cc % 8), src,
-                           ok ? 16u : 0u);
-        }
-        cp_async_commit();
-    };
-
-    // S = Q K^T for this warpgroup (its leader thread issues).
-    auto issue_s = [&](int buf, const unsigned char *kd) {
-        if (wtid == 0) {
-            tc_fence_after();
-            const uint32_t qa = smem_addr(q_s + (wg * QBUF + buf) * QBYTES), ka = smem_addr(kd);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-                umma_bf16(tmem_s, sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
-                          sdesc_sw128(ka + (kk / 4) * NK * 128 + (kk % 4) * 32, 16, 1024), idesc_s,
-                          kk > 0 ? 1u : 0u);
-            umma_commit(bar_s + wg);
-        }
-    };
-
-    // O (+)= P V, P read from tensor memory (over S).
-    auto issue_pv = [&](const unsigned char *vd, bool first) {
-        if (wtid == 0) {
-            tc_fence_after();
-            const uint32_t va = smem_addr(vd);
-            for (int kk = 0; kk < NK / 16; ++kk)
-                umma_bf16_tmem_a(tmem_o, tmem_s + kk * 8,
-                                 sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
-                                 idesc_o, (!first || kk > 0) ? 1u : 0u);
-            umma_commit(bar_o + wg);
-        }
-    };
-
-    // Warpgroup-wide bounded wait on one of its mbarriers (one thread polls).
-    auto wait_wg = [&](uint64_t *bar, uint32_t parity) -> bool {
+    auto wait_role = [&](uint64_t *bar, uint32_t parity) -> bool {
         bool ok = true;
-        if (wtid == 0) ok = mbar_wait(bar, parity, abort_flag, p.status);
-        return !named_barrier_or(wg_bar, 128, !ok || *abort_flag);
+        if ((role == 4 ? ptid : wtid) == 0) ok = mbar_wait(bar, parity, abort_flag, p.status);
+        return !named_barrier_or(role_bar, role_threads, !ok || *abort_flag);
     };
+    const uint32_t idesc_s = idesc_bf16_f32(128, NK, false);
+    const uint32_t idesc_o = idesc_bf16_f32(128, D, true);
 
-    // Softmax of this thread's row of S (sub-tile kt of chunk c): P over S in
-    // tensor memory as bf16, running max m_run / sum l_run (log2 domain).
-    auto softmax = [&](int c, int kt, float &m_run, float &l_run) {
+    // Softmax of sub-tile s of chunk c for this thread's row, one pass of 32
+    // columns at a time against the chunk's reference maximum mref (log2
+    // units).  A group more than 8 above mref raises it: P columns already
+    // written in this sub-tile, the running sum and (s > 0) O are scaled by
+    // 2^(old - new) (O once PV of the previous sub-tile has completed).
+    auto softmax_sub = [&](int c, int s, float &mref, float &lsum) -> bool {
         tc_fence_after();
         const int t = tab->t[c * TOK + tok];
-        const int lim = t - (cur_j * p.block + kt * NK);  // valid key columns: <= lim
-        const bool masked = lim < NK - 1;
-        // pass 1 over S (32 columns at a time): row max
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const int lim = t - (cur_j * p.block + s * NK);  // valid key columns: <= lim
+        const bool wmask = __any_sync(0xffffffffu, lim < NK - 1);
+        const float sc = p.scale_log2;
+        const uint64_t sc2 = f2_pack(sc, sc);
+        bool ok = true;
+        float oscale = 1.f;  // factor owed by O (the earlier sub-tiles) after reference rises
         for (int cc = 0; cc < NK / 32; ++cc) {
             uint32_t v[32];
             tmem_ld32(tmem_s + lane_addr + cc * 32, v);
             tmem_wait_ld();
-            float sv[32];
+            if (wmask) {
 #pragma unroll
-            for (int x = 0; x < 32; ++x)
-                sv[x] = (masked && cc * 32 + x > lim) ? -INFINITY : __uint_as_float(v[x]);
+                for (int x = 0; x < 32; ++x)
+                    if (cc * 32 + x > lim) v[x] = __float_as_uint(-INFINITY);
+            }
+            float g4[4] = {__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]), __uint_as_float(v[3])};
 #pragma unroll
-            for (int x = 0; x < 32; x += 8) {
-                m4[0] = fmax3(m4[0], sv[x], sv[x + 1]);
-                m4[1] = fmax3(m4[1], sv[x + 2], sv[x + 3]);
-                m4[2] = fmax3(m4[2], sv[x + 4], sv[x + 5]);
-                m4[3] = fmax3(m4[3], sv[x + 6], sv[x + 7]);
+            for (int x = 4; x < 32; x += 8) {
+                g4[0] = fmax3(g4[0], __uint_as_float(v[x]), __uint_as_float(v[x + 4]));
+                g4[1] = fmax3(g4[1], __uint_as_float(v[x + 1]), __uint_as_float(v[x + 5]));
+                g4[2] = fmax3(g4[2], __uint_as_float(v[x + 2]), __uint_as_float(v[x + 6]));
+                g4[3] = fmax3(g4[3], __uint_as_float(v[x + 3]), __uint_as_float(v[x + 7]));
             }
-        }
-        const float mt = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * p.scale_log2;
-        if (kt == 0) {
-            m_run = mt;
-            l_run = 0.f;
-        } else {
-            // online softmax across sub-tiles: rescale O only when the max
-            // grew by more than 2^8 (keeps P <= 256; exact up to rounding)
-            float alpha = 1.f;
-            bool need = false;
-            if (mt > m_run + 8.f) {
-                alpha = ex2_approx(m_run - mt);
-                m_run = mt;
-                l_run *= alpha;
-                need = true;
-            }
-            if (__any_sync(0xFFFFFFFFu, need)) {
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem_o + lane_addr + cc * 32, v);
+            const float gm = fmaxf(fmax3(g4[0], g4[1], g4[2]), g4[3]) * sc;
+            if (__any_sync(0xffffffffu, gm > mref + 8.f)) {
+                const float mnew = fmaxf(mref, gm);
+                const float f = (mref == -INFINITY || mnew == -INFINITY) ? 0.f : ex2_approx(mref - mnew);
+                if (cc > 0) tmem_wait_st();  // the P groups written so far are readable
+                for (int gq = 0; gq < cc; ++gq) {  // warp-collective; f = 1 leaves a row unchanged
+                    uint32_t w16[16];
+                    tmem_ld16(tmem_s + lane_addr + gq * 16, w16);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
-                    tmem_st32(tmem_o + lane_addr + cc * 32, v);
+                    for (int x = 0; x < 16; ++x) {
+                        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w16[x]);
+                        w16[x] = pack_bf16x2(__low2float(h) * f, __high2float(h) * f);
+                    }
+                    tmem_st16(tmem_s + lane_addr + gq * 16, w16);
                 }
-                tmem_wait_st();
+                lsum *= f;
+                oscale *= f;
+                mref = mnew;
             }
-        }
-        const float mref = m_run == -INFINITY ? 0.f : m_run;
-        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2_pack(-mref, -mref);
-        uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
-        // pass 2 over S: P = 2^(s*c - m) as bf16, written over the columns of
-        // S already consumed (32 keys -> 16 packed columns)
-        for (int cc = 0; cc < NK / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tmem_s + lane_addr + cc * 32, v);
-            tmem_wait_ld();
+            const float mr = mref == -INFINITY ? 0.f : mref;
+            const uint64_t nm2 = f2_pack(-mr, -mr);
+            uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
             uint32_t w16[16];
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
-                const float s0 = (masked && cc * 32 + 2 * x > lim) ? -INFINITY : __uint_as_float(v[2 * x]);
-                const float s1 = (masked && cc * 32 + 2 * x + 1 > lim) ? -INFINITY : __uint_as_float(v[2 * x + 1]);
                 float a0, a1;
-                f2_unpack(f2_fma(f2_pack(s0, s1), sc2, nm2), a0, a1);
-                const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * x]), __uint_as_float(v[2 * x + 1])), sc2, nm2), a0, a1);
+                const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);  // masked (-inf) columns give 0
                 if (x & 1)
                     ls2b = f2_add(ls2b, f2_pack(p0, p1));
                 else
@@ -1052,109 +1029,74 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
                 w16[x] = pack_bf16x2(p0, p1);
             }
             tmem_st16(tmem_s + lane_addr + cc * 16, w16);
+            float la0, la1, lb0, lb1;
+            f2_unpack(ls2a, la0, la1);
+            f2_unpack(ls2b, lb0, lb1);
+            lsum += (la0 + la1) + (lb0 + lb1);
         }
-        float la0, la1, lb0, lb1;
-        f2_unpack(ls2a, la0, la1);
-        f2_unpack(ls2b, lb0, lb1);
-        l_run += (la0 + la1) + (lb0 + lb1);
+        if (s > 0 && __any_sync(0xffffffffu, oscale != 1.f)) {
+            // O holds the earlier sub-tiles: once their last PV has completed,
+            // scale it to the new reference (warp-collective; 1 leaves a row)
+            bool okw = true;
+            if (lane == 0) okw = mbar_wait(bar_pv + wg, (pv_n - 1) & 1, abort_flag, p.status);
+            okw = __shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0;
+            if (!okw) ok = false;
+            tc_fence_after();
+            for (int c16 = 0; c16 < D && okw; c16 += 16) {
+                uint32_t o[16];
+                tmem_ld16(tmem_o + lane_addr + c16, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 16; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * oscale);
+                tmem_st16(tmem_o + lane_addr + c16, o);
+            }
+        }
         tmem_wait_st();
         tc_fence_before();
+        return ok;
     };
 
-    // Softmax of a whole block held in one tile (block <= 128): single pass
-    // from registers, no running max.  P over S in tensor memory as bf16.
-    auto softmax_tile = [&](int c, float &m_run, float &l_run) {
+    // epilogue warpgroup, chunk c of softmax warpgroup w (as in the resident
+    // kernel, one staging buffer).  Returns false on abort.
+    auto epilogue = [&](int c, int w) -> bool {
+        if (!wait_role(bar_o + w, eo_n[w] & 1) || !wait_role(ml_ready + w, eo_n[w] & 1)) return false;
+        ++eo_n[w];
+        const float2 ml = ml_s[w * 128 + row];
+        const float m_run = ml.x, l_run = ml.y;
+        // the bulk copies of the previous chunk have read the staging rows
+        if (g == 0) bulk_wait_read_all();
+        if (G <= 32)
+            __syncwarp();
+        else
+            named_barrier(role_bar, 128);
         tc_fence_after();
-        const int t = tab->t[c * TOK + tok];
-        const int lim = t - cur_j * p.block;  // valid key columns: <= lim
-        float sv[128];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            if (cc * 32 < NK) {
-                uint32_t v[32];
-                tmem_ld32(tmem_s + lane_addr + cc * 32, v);
-#pragma unroll
-                for (int x = 0; x < 32; ++x) sv[cc * 32 + x] = __uint_as_float(v[x]);
-            }
-        }
-        tmem_wait_ld();
-        if (lim < NK - 1) {
-#pragma unroll
-            for (int x = 0; x < 128; ++x)
-                if (x > lim) sv[x] = -INFINITY;
-        }
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int x = 0; x < 128; x += 8) {
-            if (x < NK) {
-                m4[0] = fmax3(m4[0], sv[x], sv[x + 1]);
-                m4[1] = fmax3(m4[1], sv[x + 2], sv[x + 3]);
-                m4[2] = fmax3(m4[2], sv[x + 4], sv[x + 5]);
-                m4[3] = fmax3(m4[3], sv[x + 6], sv[x + 7]);
-            }
-        }
-        m_run = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * p.scale_log2;
-        const float mref = m_run == -INFINITY ? 0.f : m_run;
-        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2_pack(-mref, -mref);
-        uint64_t ls2a = f2_pack(0.f, 0.f), ls2b = ls2a;
-#pragma unroll
-        for (int g32 = 0; g32 < 4; ++g32) {  // 32 keys -> 16 packed columns
-            if (g32 * 32 < NK) {
-                uint32_t w16[16];
-#pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    float a0, a1;
-                    f2_unpack(f2_fma(f2_pack(sv[g32 * 32 + 2 * x], sv[g32 * 32 + 2 * x + 1]), sc2, nm2), a0, a1);
-                    const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
-                    if (x & 1)
-                        ls2b = f2_add(ls2b, f2_pack(p0, p1));
-                    else
-                        ls2a = f2_add(ls2a, f2_pack(p0, p1));
-                    w16[x] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(tmem_s + lane_addr + g32 * 16, w16);
-            }
-        }
-        float la0, la1, lb0, lb1;
-        f2_unpack(ls2a, la0, la1);
-        f2_unpack(ls2b, lb0, lb1);
-        l_run = (la0 + la1) + (lb0 + lb1);
-        tmem_wait_st();
-        tc_fence_before();
-    };
-
-    // Normalised bf16 partial and its natural-log lse for chunk c.  Each
-    // thread packs its row into `stage` (the chunk's Q buffer, dead once S is
-    // done) in a token-major layout padded by 16 bytes per token (so the
-    // rows a warp writes at once spread over all banks); the first thread of
-    // each token then writes the token's G contiguous head rows of the
-    // partials with one bulk copy.  Callers wait for the copies' reads
-    // (bulk_wait_read_all) before reusing `stage`.
-    auto epilogue = [&](int c, float m_run, float l_run, unsigned char *stage) {
-        tc_fence_after();
+        const uint32_t to = tmem_base + static_cast<uint32_t>(w * 256 + 128);
         const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
         const uint64_t il2 = f2_pack(inv_l, inv_l);
         const uint32_t tok_bytes = static_cast<uint32_t>(G * D * 2 + 16);
-        unsigned char *srow = stage + tok * tok_bytes + g * (D * 2);
+        unsigned char *srow = st_s + tok * tok_bytes + g * (D * 2);
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tmem_o + lane_addr + cc * 32, v);
+        for (int c64 = 0; c64 < D; c64 += 64) {
+            uint32_t v[64];
+            tmem_ld32(to + lane_addr + c64, *reinterpret_cast<uint32_t(*)[32]>(v));
+            tmem_ld32(to + lane_addr + c64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
             tmem_wait_ld();
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint32_t w[4];
+            for (int q4 = 0; q4 < 8; ++q4) {
+                uint32_t wv[4];
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
                     float a0, a1;
                     f2_unpack(f2_mul(f2_pack(__uint_as_float(v[q4 * 8 + 2 * x]), __uint_as_float(v[q4 * 8 + 2 * x + 1])), il2), a0, a1);
-                    w[x] = pack_bf16x2(a0, a1);
+                    wv[x] = pack_bf16x2(a0, a1);
                 }
-                *reinterpret_cast<uint4 *>(srow + (cc * 4 + q4) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(srow + (c64 / 8 + q4) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
         }
+        // O and the row statistics have been read: the next chunk's PV may overwrite O
         tc_fence_before();
+        named_barrier(role_bar, 128);
+        if (wtid == 0) mbar_arrive(o_free + w);
         const int e = tab->entry[c * TOK + tok];
         if (e >= 0) {
             const long long prow = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G + g;
@@ -1162,14 +1104,17 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
         }
         fence_proxy_async_smem();
         if (G <= 32)
-            __syncwarp();  // a token's rows all belong to this warp
+            __syncwarp();
         else
-            named_barrier(wg_bar, 128);
-        if (g == 0 && e >= 0) {
-            const long long prow0 = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G;
-            bulk_store(p.part_o + prow0 * D, stage + tok * tok_bytes, static_cast<uint32_t>(G * D * 2));
+            named_barrier(role_bar, 128);
+        if (g == 0) {
+            if (e >= 0) {
+                const long long prow0 = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G;
+                bulk_store_hint(p.part_o + prow0 * D, st_s + tok * tok_bytes, static_cast<uint32_t>(G * D * 2), pol_first);
+            }
             bulk_commit();
         }
+        return true;
     };
 
     while (true) {
@@ -1180,18 +1125,12 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
         const int hk = w / n_items;
         const AttnItem item = p.items[w - hk * n_items];
         const int b = item.pair / p.N, j = item.pair - b * p.N;
-        cur_b = b;
         cur_j = j;
         cur_hk = hk;
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
-        // chunks of this warpgroup: c = wg, wg + 2, ...
-        const int my_chunks = n_chunks > wg ? (n_chunks - wg + 1) / 2 : 0;
 
-        if (tid == 0) issue_kv(b, j, hk, 0);
-        // token table of the item: coalesced loads of its list entries and
-        // one division per token (tokens past the list end stay invalid)
         for (int i = tid; i < n_chunks * TOK; i += blockDim.x) {
             int e = -1, t = -1;
             int qo16 = 0;
@@ -1213,103 +1152,187 @@ __global__ void __launch_bounds__(256, 1) prefill_attn_kernel(
         }
         __syncthreads();
 
-        if (!streamed) {
-            // ---- K/V resident for the whole item; each warpgroup pipelines its
-            // chunks: S(c+1) is issued before the epilogue of c.
-            const unsigned char *kd = kv_s, *vd = kv_s + kv_tile;
-            const int n = my_chunks;
-            if (n > 0) gather(0, wg);
-            for (int ci = 0; ci < n; ++ci) {
-                const int c = wg + 2 * ci, buf = ci & 1;
-                cp_async_wait_all();
+        if (role == 4) {
+            // ---- producers: chunk c goes to softmax warpgroup c & 1, two halves per tile
+            const int cc = ptid % PPR, r0 = ptid / PPR;
+            const uint4 *qcol = reinterpret_cast<const uint4 *>(p.q) + cc;
+            for (int c = 0; c < n_chunks && !aborted; ++c) {
+                const int x = c & 1, ci = c >> 1;
+                unsigned char *dst = q_s + x * QT + (cc / 8) * kRegionBytes;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    uint4 v[NLDH];
+#pragma unroll
+                    for (int k = 0; k < NLDH; ++k) {
+                        const int r = 64 * h + r0 + k * RSTEP;
+                        if (k < NLDH - 1 || r < 64 * h + 64)  // padding rows read row 0 (output dropped)
+                            v[k] = ld_nc_na_16_hint(qcol + tab->qo16[c * TOK + (r >> p.log2G)] + (r & (G - 1)) * PPR,
+                                                    pol_last);
+                    }
+                    if (h == 0 && ci >= 1) {  // the last S of the warpgroup's previous chunk has read the tile
+                        if (!wait_role(q_free + x, pf[x] & 1)) {
+                            aborted = true;
+                            break;
+                        }
+                        ++pf[x];
+                    }
+#pragma unroll
+                    for (int k = 0; k < NLDH; ++k) {
+                        const int r = 64 * h + r0 + k * RSTEP;
+                        if (k < NLDH - 1 || r < 64 * h + 64)
+                            *reinterpret_cast<uint4 *>(dst + sw128_offset(r, cc % 8)) = v[k];
+                    }
+                    asm volatile("" ::: "memory");  // one half's registers at a time
+                }
+                if (aborted) break;
                 fence_proxy_async_smem();
-                if (ci == 0) {
-                    if (!wait_wg(kvfull, item_n & 1)) { aborted = true; break; }
-                } else {
-                    named_barrier(wg_bar, 128);
-                }
-                issue_s(buf, kd);
-                // next chunk's Q into the other buffer: its S finished a chunk ago
-                // and its staged partial has been read by the bulk copies
-                if (ci + 1 < n) {
-                    bulk_wait_read_all();
-                    named_barrier(wg_bar, 128);
-                    gather(buf ^ 1, c + 2);
-                }
-                if (!wait_wg(bar_s + wg, s_n & 1)) { aborted = true; break; }
-                ++s_n;
-                float m_run, l_run;
-                softmax_tile(c, m_run, l_run);
-                named_barrier(wg_bar, 128);
-                issue_pv(vd, true);
-                if (!wait_wg(bar_o + wg, o_n & 1)) { aborted = true; break; }
-                ++o_n;
-                epilogue(c, m_run, l_run, q_s + (wg * QBUF + buf) * QBYTES);
+                named_barrier(role_bar, NPROD);
+                if (ptid == 0) mbar_arrive(q_ready + x);
             }
-        } else {
-            // ---- K/V streamed in sub-tiles (double-buffered); both warpgroups
-            // walk (chunk pair, sub-tile) in lockstep with an online softmax.
-            const int pairs = (n_chunks + 1) / 2;
-            const int n_steps = pairs * p.NS;
-            float m_run = -INFINITY, l_run = 0.f;
-            if (my_chunks > 0) gather(0, wg);
-            for (int step = 0; step < n_steps; ++step) {
-                const int ci = step / p.NS, kt = step % p.NS;
-                const int c = wg + 2 * ci;
-                const bool active = c < n_chunks;
-                if (kt == 0 && active && ci > 0) {
-                    bulk_wait_read_all();  // staged partial of the previous chunk read out
-                    named_barrier(wg_bar, 128);
-                    gather(0, c);
-                }
-                if (kt == 0) cp_async_wait_all();
-                fence_proxy_async_smem();
-                const uint32_t st = kv_use % KVST;
+        } else if (role == 3) {
+            // ---- K/V streaming and MMA issue (one thread)
+            if (lane == 0) {
+                const int R = (n_chunks + 1) / 2;              // rounds (chunk pairs)
+                const int nr[2] = {R, n_chunks / 2};           // rounds with a chunk, per warpgroup
+                const int ntiles = R * NS * 2;                 // K_0 V_0 K_1 V_1 ... per round
+                const uint32_t t0 = gt;                        // first tile of the item (global count)
+                int tl = 0;                                    // tiles of the item issued
+                int readers[kKvSlots] = {0, 0, 0};
+                int rr[2] = {0, 0}, ss[2] = {0, 0}, act[2] = {0, 0};  // act: 0 = S next, 1 = PV next
                 bool ok = true;
-                if (tid == 0) ok = mbar_wait(kvfull + st, (kv_use / KVST) & 1, abort_flag, p.status);
-                ++kv_use;
-                if (__syncthreads_or(!ok || *abort_flag)) { aborted = true; break; }
-                if (tid == 0 && step + 1 < n_steps) issue_kv(b, j, hk, (step + 1) % p.NS);
-                const unsigned char *kd = kv_s + st * 2 * kv_tile;
-                const unsigned char *vd = kd + kv_tile;
-                if (active) issue_s(0, kd);
-                ok = true;
-                if (active && wtid == 0) ok = mbar_wait(bar_s + wg, s_n & 1, abort_flag, p.status);
-                if (active) ++s_n;
-                if (__syncthreads_or(!ok || *abort_flag)) { aborted = true; break; }
-                if (active) softmax(c, kt, m_run, l_run);
-                named_barrier(wg_bar, 128);
-                if (active) issue_pv(vd, kt == 0);
-                ok = true;
-                if (active && wtid == 0) ok = mbar_wait(bar_o + wg, o_n & 1, abort_flag, p.status);
-                if (active) ++o_n;
-                if (__syncthreads_or(!ok || *abort_flag)) { aborted = true; break; }
-                if (active && kt == p.NS - 1) {
-                    epilogue(c, m_run, l_run, q_s + wg * QBUF * QBYTES);
-                    m_run = -INFINITY;
-                    l_run = 0.f;
+                uint64_t tw = global_timer_ns();
+                auto tile_in = [&](int ti) -> bool {  // tile ti of the item has landed
+                    if (ti >= tl) return false;
+                    const uint32_t gg = t0 + static_cast<uint32_t>(ti);
+                    return mbar_test(kvfull + gg % kKvSlots, (gg / kKvSlots) & 1);
+                };
+                auto release = [&](int ti) {  // one reader of tile ti has issued its MMA
+                    const uint32_t sl = (t0 + static_cast<uint32_t>(ti)) % kKvSlots;
+                    if (--readers[sl] == 0) umma_commit(slot_free + sl);
+                };
+                while (ok && (rr[0] < nr[0] || rr[1] < nr[1])) {
+                    bool progress = false;
+                    // refill: the next tile once its slot's previous tile is released
+                    if (tl < ntiles) {
+                        const uint32_t gg = t0 + static_cast<uint32_t>(tl);
+                        const uint32_t sl = gg % kKvSlots;
+                        if (gg < kKvSlots || mbar_test(slot_free + sl, ((gg / kKvSlots) - 1) & 1)) {
+                            const int pair = tl >> 1, s = pair % NS, r = pair / NS;
+                            readers[sl] = (2 * r + 1 < n_chunks) ? 2 : 1;
+                            unsigned char *dst = kv_s + sl * kv_tile;
+                            mbar_arrive_expect_tx(kvfull + sl, kv_tile);
+                            const int z = b * p.T + j * p.block + s * NK;
+                            for (int rg = 0; rg < DREG; ++rg)
+                                tma_load_3d(dst + rg * NK * 128, (tl & 1) ? &tm_v : &tm_k, kvfull + sl, rg * 64, hk, z);
+                            ++tl;
+                            progress = true;
+                        }
+                    }
+                    for (int x = 0; x < 2; ++x) {
+                        if (rr[x] >= nr[x]) continue;
+                        const int tK = (rr[x] * NS + ss[x]) * 2;
+                        const uint32_t ts = tmem_base + static_cast<uint32_t>(x * 256);
+                        if (act[x] == 0) {
+                            if (!tile_in(tK)) continue;
+                            if (ss[x] == 0 && !mbar_test(q_ready + x, mq[x] & 1)) continue;
+                            if ((rr[x] > 0 || ss[x] > 0) && !mbar_test(bar_pv + x, (mp[x] - 1) & 1)) continue;
+                            tc_fence_after();
+                            const uint32_t qa = smem_addr(q_s + x * QT);
+                            const uint32_t ka = smem_addr(kv_s + ((t0 + tK) % kKvSlots) * kv_tile);
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                umma_bf16(ts, sdesc_sw128(qa + (kk / 4) * kRegionBytes + (kk % 4) * 32, 16, 1024),
+                                          sdesc_sw128(ka + (kk / 4) * NK * 128 + (kk % 4) * 32, 16, 1024),
+                                          idesc_s, kk > 0 ? 1u : 0u);
+                            umma_commit(bar_s + x);
+                            release(tK);
+                            if (ss[x] == 0) ++mq[x];
+                            act[x] = 1;
+                        } else {
+                            if (!mbar_test(p_ready + x, mp[x] & 1)) continue;
+                            if (!tile_in(tK + 1)) continue;
+                            tc_fence_after();
+                            const uint32_t va = smem_addr(kv_s + ((t0 + tK + 1) % kKvSlots) * kv_tile);
+                            for (int kk = 0; kk < NK / 16; ++kk)
+                                umma_bf16_tmem_a(ts + 128, ts + kk * 8,
+                                                 sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
+                                                 idesc_o, (ss[x] > 0 || kk > 0) ? 1u : 0u);
+                            umma_commit(bar_pv + x);
+                            if (ss[x] == NS - 1) umma_commit(bar_o + x);
+                            release(tK + 1);
+                            ++mp[x];
+                            act[x] = 0;
+                            if (++ss[x] == NS) {
+                                ss[x] = 0;
+                                ++rr[x];
+                            }
+                        }
+                        progress = true;
+                    }
+                    if (progress) {
+                        tw = global_timer_ns();
+                    } else if (*abort_flag) {
+                        ok = false;
+                    } else if (global_timer_ns() - tw > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        atomicOr(p.status, kDevTimeout);
+                        ok = false;
+                    }
                 }
+                if (!ok) {
+                    aborted = true;
+                    // copies still in flight land before the CTA moves on
+                    for (int ti = tl > kKvSlots ? tl - kKvSlots : 0; ti < tl; ++ti) {
+                        const uint32_t gg = t0 + static_cast<uint32_t>(ti);
+                        mbar_drain(kvfull + gg % kKvSlots, (gg / kKvSlots) & 1);
+                    }
+                }
+                gt = t0 + static_cast<uint32_t>(tl);
+            }
+        } else if (role == 2) {
+            // ---- epilogue warpgroup: every chunk of the item in order
+            for (int c = 0; c < n_chunks; ++c)
+                if (!epilogue(c, c & 1)) {
+                    aborted = true;
+                    break;
+                }
+        } else {
+            // ---- softmax warpgroup: chunks c = wg + 2r, every sub-tile of each
+            const int n = (n_chunks + 1 - wg) / 2;
+            for (int r = 0; r < n && !aborted; ++r) {
+                const int c = wg + 2 * r;
+                float mref = -INFINITY, lsum = 0.f;
+                for (int s = 0; s < NS; ++s) {
+                    if (!wait_role(bar_s + wg, s_n & 1)) { aborted = true; break; }
+                    ++s_n;
+                    if (wtid == 0 && s == NS - 1 && r + 1 < n) mbar_arrive(q_free + wg);
+                    const bool sok = softmax_sub(c, s, mref, lsum);
+                    // the epilogue warpgroup has read O of this warpgroup's previous chunk
+                    if (s == 0 && och > 0 && !wait_role(o_free + wg, (och - 1) & 1)) { aborted = true; break; }
+                    if (s == NS - 1) ml_s[wg * 128 + row] = make_float2(mref, lsum);
+                    if (named_barrier_or(role_bar, 128, !sok)) { aborted = true; break; }
+                    if (wtid == 0) {
+                        if (s == NS - 1) mbar_arrive(ml_ready + wg);
+                        mbar_arrive(p_ready + wg);
+                    }
+                    ++pv_n;
+                }
+                ++och;
             }
         }
         ++item_n;
-        bulk_wait_read_all();  // staged partials read before the buffers are reused
-        // both warpgroups done with this item's K/V, Q buffers and table
         if (__syncthreads_or(aborted)) {
             aborted = true;
             break;
         }
     }
     __syncthreads();
-    if (aborted && tid == 0) {
-        for (int s2 = 0; s2 < 2; ++s2)
-            if (armed_parity[s2] >= 0) mbar_drain(kvfull + s2, static_cast<uint32_t>(armed_parity[s2]));
-    }
-    cp_async_wait_all();
     bulk_wait_all();
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(*tmem_slot, 512);
+    if (warp == 0) tmem_dealloc(tmem_base, 512);
 }
+
 
 }  // namespace
 
@@ -1374,7 +1397,8 @@ size_t prefill_attn_smem_bytes(const Shape &sh) {
     const size_t q = static_cast<size_t>(sh.d / 64) * kRegionBytes + 2048;
     if (NS == 1)  // resident kernel: K/V, two Q tiles, two staging buffers, row statistics
         return 1024 + 2 * kv_tile + 2 * (q - 2048) + 2 * q + 2 * 128 * 8 + sizeof(ItemRows) + 160 + 32;
-    return 1024 + KVST * 2 * kv_tile + 2 * QBUF * q + sizeof(ItemRows) + 160 + 32;
+    // streamed kernel: K/V tile slots, two Q tiles, one staging buffer, row statistics
+    return 1024 + kKvSlots * kv_tile + 2 * (q - 2048) + q + 2 * 128 * 8 + sizeof(ItemRows) + 192 + 32;
 }
 
 int prefill_attn_rows_per_item(int G) {
@@ -1421,8 +1445,8 @@ cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const 
         if (sh.d == 128) MSA_LAUNCH(prefill_attn_resident_kernel<128>, kResidentThreads);
         else MSA_LAUNCH(prefill_attn_resident_kernel<64>, kResidentThreads);
     } else {
-        if (sh.d == 128) MSA_LAUNCH(prefill_attn_kernel<128>, 256);
-        else MSA_LAUNCH(prefill_attn_kernel<64>, 256);
+        if (sh.d == 128) MSA_LAUNCH(prefill_attn_streamed_kernel<128>, kStreamedThreads);
+        else MSA_LAUNCH(prefill_attn_streamed_kernel<64>, kStreamedThreads);
     }
 #undef MSA_LAUNCH
     return cudaGetLastError();
