@@ -429,7 +429,7 @@ template <typename PT, int D>
 __global__ void __launch_bounds__(256) lse_combine_kernel(
     const PT *__restrict__ part_o, const float *__restrict__ part_lse,
     const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
-    int K, int S, int HG) {
+    int K, int S, int HG, int G) {
     constexpr int VEC = 16 / sizeof(PT);  // elements per 16-byte load
     constexpr int NV = D / VEC;           // 16-byte loads per head row
     extern __shared__ float wsm[];        // [P][HG] weights, then [HG] LSE
@@ -471,7 +471,12 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
         float acc[VEC];
 #pragma unroll
         for (int x = 0; x < VEC; ++x) acc[x] = 0.f;
-        const PT *src = part_o + ((row * K) * S * Hq + h0 + hh) * static_cast<long long>(D) + c;
+        // G > 0: the prefill kernels store 16-byte piece q of a head row with
+        // head index g inside its kv group at q ^ ((g * max(1, 8 / G)) & 7)
+        const int gh = G > 0 ? ((h0 + hh) & (G - 1)) : 0;
+        const int rot = G > 0 ? (gh * (G >= 8 ? 1 : 8 / G)) & 7 : 0;
+        const int cr = ((c / VEC) ^ rot) * VEC;
+        const PT *src = part_o + ((row * K) * S * Hq + h0 + hh) * static_cast<long long>(D) + cr;
         const long long pstride = static_cast<long long>(Hq) * D;  // between consecutive partials
 #pragma unroll 4
         for (int pp = 0; pp < P; ++pp) {
@@ -876,7 +881,8 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
         cudaFuncSetAttribute(lse_combine_kernel<PT, DD>,                                         \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
         lse_combine_kernel<PT, DD><<<grid, threads, smem, st>>>(                                 \
-            static_cast<const PT *>(part_o), part_lse, ids, out, lse, sh.Hq, sh.K, S, HG);       \
+            static_cast<const PT *>(part_o), part_lse, ids, out, lse, sh.Hq, sh.K, S, HG,        \
+            part_bf16 ? sh.G : 0);                                                               \
     } while (0)
     if (part_bf16) {
         if (sh.d == 128) MSA_COMBINE(__nv_bfloat16, 128); else MSA_COMBINE(__nv_bfloat16, 64);

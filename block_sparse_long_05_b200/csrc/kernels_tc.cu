@@ -667,6 +667,9 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         const uint64_t il2 = f2_pack(inv_l, inv_l);
         const uint32_t tok_bytes = static_cast<uint32_t>(G * D * 2 + 16);
         unsigned char *srow = stage + tok * tok_bytes + g * (D * 2);
+        // 16-byte piece q of this head row is stored at q ^ prot (the partial
+        // layout the combine reads), so a phase's 8 lanes hit 8 bank groups
+        const int prot = (g * (G >= 8 ? 1 : 8 / G)) & 7;
 #pragma unroll
         for (int c64 = 0; c64 < D; c64 += 64) {
             uint32_t v[64];
@@ -682,7 +685,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
                     f2_unpack(f2_mul(f2_pack(__uint_as_float(v[q4 * 8 + 2 * x]), __uint_as_float(v[q4 * 8 + 2 * x + 1])), il2), a0, a1);
                     wv[x] = pack_bf16x2(a0, a1);
                 }
-                *reinterpret_cast<uint4 *>(srow + (c64 / 8 + q4) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                *reinterpret_cast<uint4 *>(srow + ((c64 / 8 + q4) ^ prot) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
         }
         // O and the row statistics have been read: the warpgroup may issue its next PV
@@ -1075,6 +1078,9 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
         const uint64_t il2 = f2_pack(inv_l, inv_l);
         const uint32_t tok_bytes = static_cast<uint32_t>(G * D * 2 + 16);
         unsigned char *srow = st_s + tok * tok_bytes + g * (D * 2);
+        // 16-byte piece q of this head row is stored at q ^ prot (the partial
+        // layout the combine reads), so a phase's 8 lanes hit 8 bank groups
+        const int prot = (g * (G >= 8 ? 1 : 8 / G)) & 7;
 #pragma unroll
         for (int c64 = 0; c64 < D; c64 += 64) {
             uint32_t v[64];
@@ -1090,7 +1096,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
                     f2_unpack(f2_mul(f2_pack(__uint_as_float(v[q4 * 8 + 2 * x]), __uint_as_float(v[q4 * 8 + 2 * x + 1])), il2), a0, a1);
                     wv[x] = pack_bf16x2(a0, a1);
                 }
-                *reinterpret_cast<uint4 *>(srow + (c64 / 8 + q4) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                *reinterpret_cast<uint4 *>(srow + ((c64 / 8 + q4) ^ prot) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
         }
         // O and the row statistics have been read: the next chunk's PV may overwrite O
