@@ -645,14 +645,21 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         tc_fence_before();
     };
 
-    // epilogue warpgroup, chunk c of softmax warpgroup w: normalised bf16
-    // partial rows of O staged token-major (16-byte pad per token), one bulk
-    // copy per token; lse stored directly.  Returns false on abort.
+    // lse of this thread's row of chunk c (softmax warpgroup), natural log
+    auto store_lse = [&](int c, float m_run, float l_run) {
+        const int e = tab->entry[c * TOK + tok];
+        if (e >= 0) {
+            const long long prow = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G + g;
+            p.part_lse[prow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2f : -INFINITY;
+        }
+    };
+    // epilogue warpgroup, chunk c of softmax warpgroup w: partial rows of O
+    // scaled by 1/l, as bf16, staged token-major (16-byte pad per token), one
+    // bulk copy per token.  Returns false on abort.
     auto epilogue = [&](int c, int w) -> bool {
         if (!wait_role(bar_o + w, eo_n[w] & 1) || !wait_role(ml_ready + w, eo_n[w] & 1)) return false;
         ++eo_n[w];
-        const float2 ml = ml_s[w * 128 + row];
-        const float m_run = ml.x, l_run = ml.y;
+        const float inv_l = ml_s[w * 128 + row].y;  // 1 / l, or 0 for a row without keys
         unsigned char *stage = st_s + (ec_n & 1) * STB;
         ++ec_n;
         // the bulk copies that last read this staging buffer (two chunks ago) are done
@@ -663,7 +670,6 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
             named_barrier(role_bar, 128);
         tc_fence_after();
         const uint32_t to = tmem_base + static_cast<uint32_t>(w * 256 + 128);
-        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
         const uint64_t il2 = f2_pack(inv_l, inv_l);
         const uint32_t tok_bytes = static_cast<uint32_t>(G * D * 2 + 16);
         unsigned char *srow = stage + tok * tok_bytes + g * (D * 2);
@@ -693,10 +699,6 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         named_barrier(role_bar, 128);
         if (wtid == 0) mbar_arrive(o_free + w);
         const int e = tab->entry[c * TOK + tok];
-        if (e >= 0) {
-            const long long prow = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G + g;
-            p.part_lse[prow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
-        }
         fence_proxy_async_smem();
         if (G <= 32)
             __syncwarp();
@@ -812,9 +814,10 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
                 if (wtid == 0 && ci + 1 < n) mbar_arrive(q_free + wg);
                 float m_run, l_run;
                 softmax_tile(c, m_run, l_run);
-                // the epilogue warpgroup has read O and (m, l) of the previous PV
+                store_lse(c, m_run, l_run);
+                // the epilogue warpgroup has read O and 1/l of the previous PV
                 if (pv_n > 0 && !wait_role(o_free + wg, (pv_n - 1) & 1)) { aborted = true; break; }
-                ml_s[wg * 128 + row] = make_float2(m_run, l_run);
+                ml_s[wg * 128 + row] = make_float2(m_run, l_run > 0.f ? 1.f / l_run : 0.f);
                 named_barrier(role_bar, 128);
                 if (wtid == 0) {
                     mbar_arrive(ml_ready + wg);
