@@ -391,23 +391,19 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
 // ===========================================================================
 // Prefill attention (KV-block-outer).
 //
-// One CTA per SM, 256 threads = two warpgroups (WG0 = warps 0-3, WG1 = warps
-// 4-7).  A work item is (kv head hk, sequence b, block j, slice of the block's
-// hit list).  Thread 0 TMA-loads K_j and V_j of head hk into shared memory
-// once per item (block <= 128) or per 128-key sub-tile (block > 128).  The
-// item's hit list is cut into 128-row chunks (128/G tokens x G heads); the
-// two warpgroups take alternate chunks and run them independently, so one
-// warpgroup's softmax overlaps the other's tensor-core work:
-//   gather Q rows (cp.async, double-buffered per warpgroup)
+// A work item is (kv head hk, sequence b, block j, slice of the block's hit
+// list): the queries that selected block j, each with its G heads of kv head
+// hk.  The list is cut into 128-row chunks (128/G tokens x G heads); every
+// chunk yields, per row, the softmax partial over the keys of block j (keys
+// after the query position masked):
 //   S = Q K^T          (tcgen05, S in tensor memory)
-//   P = exp2(S*c - m)  (registers; P written back over S as bf16)
+//   P = 2^(S*c - m)    (registers; bf16 P written back over S)
 //   O = P V            (tcgen05, A operand read from tensor memory)
 //   partial row: O / l in bf16, lse = ln(l) + m  (per query, slot and head)
-// Tensor memory: WG w owns columns [256w, 256w+256): S/P at +0, O at +128.
-// With block > 128 the warpgroups walk the sub-tiles in lockstep (K/V
-// double-buffered) with an online softmax; the O rescale is only done when
-// the running max grows by more than 2^8, which keeps P <= 256 and the
-// result exact up to rounding.
+// and a later kernel merges the K partials of each row by their lse.  Blocks
+// of at most 128 keys keep K_j and V_j resident per item (resident kernel);
+// longer blocks stream them in 128-key sub-tiles (streamed kernel).  Work
+// items are taken from a global queue by persistent CTAs, one per SM.
 // ===========================================================================
 struct AttnParams {
     const __nv_bfloat16 *q;
