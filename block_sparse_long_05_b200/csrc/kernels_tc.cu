@@ -174,7 +174,7 @@ struct IndexParams {
     int Bt, n_q, T, block, K, n_qt, n_items;
 };
 
-constexpr int kIdxStages = 4;
+constexpr int kIdxStages = 3;
 
 __device__ __forceinline__ int snake_item(int it, int cta, int ncta) {
     return (it & 1) ? it * ncta + (ncta - 1 - cta) : it * ncta + cta;
@@ -204,12 +204,14 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     IndexParams p) {
     constexpr int NREG = D_IDX / 64;
-    constexpr uint32_t TILE = NREG * kRegionBytes;
+    constexpr uint32_t TILE = NREG * kRegionBytes;         // Q tile: 128 rows
+    constexpr uint32_t KREG = kIdxKeys * 128;               // one 64-column region of a key tile
+    constexpr uint32_t KTILE = NREG * KREG;                 // key tile: kIdxKeys rows
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = align1024(smem_raw);
     unsigned char *q_s = base;
-    unsigned char *k_s = base + TILE;  // kIdxStages tiles
-    uint64_t *bars = reinterpret_cast<uint64_t *>(k_s + kIdxStages * TILE);
+    unsigned char *k_s = base + TILE;  // kIdxStages key tiles
+    uint64_t *bars = reinterpret_cast<uint64_t *>(k_s + kIdxStages * KTILE);
     uint64_t *kfull = bars;
     uint64_t *kempty = bars + kIdxStages;
     uint64_t *qfull = bars + 2 * kIdxStages;
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 2 * kIdxKeys);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
                 const int qt = p.n_qt - 1 - idx / p.Bt, b = idx % p.Bt;
                 const int i_last = min(qt * 128 + 127, p.n_q - 1);
                 const int own_max = (p.T - p.n_q + i_last) / B;
-                const int n_sub = (own_max * B + 127) / 128;
+                const int n_sub = (own_max * B + kIdxKeys - 1) / kIdxKeys;
                 if (!mbar_wait(qempty, (it & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
                 mbar_arrive_expect_tx(qfull, TILE);
                 for (int r = 0; r < NREG; ++r)
@@ -266,11 +268,11 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
                 for (int s = 0; s < n_sub; ++s, ++n) {
                     const uint32_t st = n % kIdxStages, rd = n / kIdxStages;
                     if (!mbar_wait(kempty + st, (rd & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
-                    mbar_arrive_expect_tx(kfull + st, TILE);
+                    mbar_arrive_expect_tx(kfull + st, KTILE);
                     armed[st] = static_cast<int>(rd & 1);
                     for (int r = 0; r < NREG; ++r)
-                        tma_load_2d(k_s + st * TILE + r * kRegionBytes, &tm_k, kfull + st, r * 64,
-                                    b * p.T + s * 128);
+                        tma_load_2d(k_s + st * KTILE + r * KREG, &tm_k, kfull + st, r * 64,
+                                    b * p.T + s * kIdxKeys);
                 }
             }
             if (*abort_flag) {  // drain this CTA's copies still in flight
@@ -280,7 +282,7 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, 128, false);
+            const uint32_t idesc = idesc_bf16_f32(128, kIdxKeys, false);
             uint32_t n = 0, acc_n = 0;
             bool ok = true;
             for (int it = 0; ok; ++it) {
@@ -289,7 +291,7 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
                 const int qt = p.n_qt - 1 - idx / p.Bt;
                 const int i_last = min(qt * 128 + 127, p.n_q - 1);
                 const int own_max = (p.T - p.n_q + i_last) / B;
-                const int n_sub = (own_max * B + 127) / 128;
+                const int n_sub = (own_max * B + kIdxKeys - 1) / kIdxKeys;
                 if (!mbar_wait(qfull, it & 1, abort_flag, p.status)) break;
                 for (int s = 0; s < n_sub; ++s, ++n, ++acc_n) {
                     const uint32_t st = n % kIdxStages, rd = n / kIdxStages;
@@ -297,12 +299,12 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
                     if (!mbar_wait(kfull + st, rd & 1, abort_flag, p.status)) { ok = false; break; }
                     if (!mbar_wait(tempty + acc, (ar & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t qa = smem_addr(q_s), ka = smem_addr(k_s + st * TILE);
+                    const uint32_t qa = smem_addr(q_s), ka = smem_addr(k_s + st * KTILE);
 #pragma unroll
                     for (int kk = 0; kk < D_IDX / 16; ++kk) {
-                        const uint32_t off = (kk / 4) * kRegionBytes + (kk % 4) * 32;
-                        umma_bf16(tmem + acc * 128, sdesc_sw128(qa + off, 16, 1024),
-                                  sdesc_sw128(ka + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                        const uint32_t koff = (kk % 4) * 32;
+                        umma_bf16(tmem + acc * kIdxKeys, sdesc_sw128(qa + (kk / 4) * kRegionBytes + koff, 16, 1024),
+                                  sdesc_sw128(ka + (kk / 4) * KREG + koff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(kempty + st);
                     umma_commit(tfull + acc);
@@ -323,7 +325,7 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
             const int qt = p.n_qt - 1 - idx / p.Bt, b = idx % p.Bt;
             const int i_last = min(qt * 128 + 127, p.n_q - 1);
             const int own_max = (p.T - p.n_q + i_last) / B;
-            const int n_sub = (own_max * B + 127) / 128;
+            const int n_sub = (own_max * B + kIdxKeys - 1) / kIdxKeys;
             const int i = qt * 128 + row;
             const bool valid = i < p.n_q;
             const int own = valid ? (p.T - p.n_q + i) / B : 0;
@@ -340,16 +342,16 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
                 if (!mbar_wait(tfull + acc, ar & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < kIdxKeys / 32; ++c) {
                     uint32_t v[32];
-                    tmem_ld32(tmem + lane_addr + acc * 128 + c * 32, v);
+                    tmem_ld32(tmem + lane_addr + acc * kIdxKeys + c * 32, v);
                     tmem_wait_ld();
                     // block >= 32 and 32 | block: a 32-column chunk lies in one block
                     float m = -FLT_MAX;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) m = fmaxf(m, __uint_as_float(v[e]));
                     bm = fmaxf(bm, m);
-                    const int col_end = s * 128 + c * 32 + 32;
+                    const int col_end = s * kIdxKeys + c * 32 + 32;
                     if (col_end % B == 0) {
                         const int j = col_end / B - 1;
                         if (j < own) topk_insert<CAP>(ts, tj, bm, j);
@@ -385,7 +387,7 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tmem, 256);
+    if (warp == 1) tmem_dealloc(tmem, 2 * kIdxKeys);
 }
 
 // ===========================================================================
@@ -1357,7 +1359,7 @@ cudaError_t launch_selftest_umma(const CUtensorMap &tm_a, const CUtensorMap &tm_
 }
 
 size_t prefill_index_smem_bytes(int d_idx) {
-    return 1024 + static_cast<size_t>(1 + kIdxStages) * (d_idx / 64) * kRegionBytes + 256;
+    return 1024 + static_cast<size_t>(d_idx / 64) * (kRegionBytes + kIdxStages * kIdxKeys * 128) + 256;
 }
 
 template <int D_IDX, int CAP>

@@ -197,8 +197,9 @@ msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids,
     const cuuint64_t dq[2] = {static_cast<cuuint64_t>(d_idx), static_cast<cuuint64_t>(Bt) * n_q};
     const cuuint64_t dk[2] = {static_cast<cuuint64_t>(d_idx), static_cast<cuuint64_t>(Bt) * T};
     const cuuint64_t str[1] = {static_cast<cuuint64_t>(d_idx) * 2};
-    const cuuint32_t box[2] = {64, 128};
-    if (!make_tmap(&tq, q_idx, 2, dq, str, box) || !make_tmap(&tk, k_idx, 2, dk, str, box))
+    const cuuint32_t qbox[2] = {64, 128};                              // 128-query tile
+    const cuuint32_t kbox[2] = {64, static_cast<cuuint32_t>(kIdxKeys)};  // key tile
+    if (!make_tmap(&tq, q_idx, 2, dq, str, qbox) || !make_tmap(&tk, k_idx, 2, dk, str, kbox))
         return MSA_ERR_CUDA;
     mark(ev, 0, true, st);
     const cudaError_t e = launch_prefill_index(sh, tq, tk, ids, status, sms, st);

@@ -15,6 +15,7 @@ constexpr int kMaxK = 32;          // top-K capacity of the register lists
 constexpr int kMaxBlocksPrefill = 8192;  // N limit (inversion histograms, decode select)
 constexpr int kInvRows = 128;      // query rows per inversion chunk (4 warps x 32)
 constexpr int kDecodeKeys = 64;    // keys per split of the decode attention kernel
+constexpr int kIdxKeys = 256;      // keys per tile of the prefill index kernel (one MMA N)
 
 // Problem sizes of one call (host-validated).
 struct Shape {
