@@ -21,7 +21,7 @@
  *        (the inversion of the per-query selection).
  *        Section 3.3: decode = one query, the newest position.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - K counts the own block; ties in the index score go to the lower block
  *     index; ids are emitted ascending and padded with -1.
  *   - The own block is forced, the other candidates are blocks j < own(t).
