@@ -1,6 +1,7 @@
 // ptx_sm100.cuh -- inline-PTX wrappers for sm_100a: mbarriers with bounded
-// waits, TMA tile loads (no cluster multicast), cp.async gathers, and the
-// tcgen05 tensor-core / tensor-memory instructions.
+// waits, TMA tile loads (no cluster multicast), bulk copies, cache-policy
+// loads, packed fp32 arithmetic, and the tcgen05 tensor-core / tensor-memory
+// instructions.
 //
 // Every wait in this library is bounded: a wait that exceeds kWaitLimitNs of
 // wall time raises an abort flag in shared memory and an error bit in the
@@ -119,14 +120,9 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
-// Bulk (non-tensor) copy shared -> global, tracked by bulk groups.  Both
-// addresses 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
-                 "r"(smem_addr(ssrc)), "r"(bytes)
-                 : "memory");
-}
-// bulk_store with an L2 eviction policy.
+// Bulk (non-tensor) copy shared -> global with an L2 eviction policy,
+// tracked by bulk groups.  Both addresses 16-byte aligned, size a multiple
+// of 16.
 __device__ __forceinline__ void bulk_store_hint(void *gdst, const void *ssrc, uint32_t bytes, uint64_t pol) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;"
                  ::"l"(gdst), "r"(smem_addr(ssrc)), "r"(bytes), "l"(pol)
@@ -148,16 +144,6 @@ __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
-// 16-byte read-only global load that does not allocate in L1 (streams of
-// gathered rows that are used once per SM).
-__device__ __forceinline__ uint4 ld_nc_na_16(const void *src) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(src));
-    return v;
-}
-
 // L2 eviction-priority policies for the .L2::cache_hint forms below.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t pol;
@@ -169,37 +155,14 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
-// ld_nc_na_16 with an L2 eviction policy.
+// 16-byte read-only global load that does not allocate in L1, with an L2
+// eviction policy (gathered rows, used once per SM).
 __device__ __forceinline__ uint4 ld_nc_na_16_hint(const void *src, uint64_t pol) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(src), "l"(pol));
     return v;
-}
-
-// ---------------------------------------------------------------- cp.async
-// 16-byte global->shared copy; src_bytes = 0 fills the destination with zeros.
-__device__ __forceinline__ void cp_async_16(void *dst, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)),
-                 "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-// Same, allocating in L1 (lets the L1 merge a warp's pieces of one line).
-__device__ __forceinline__ void cp_async_16_ca(void *dst, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)),
-                 "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
-// wait until at most one committed group is still pending
-__device__ __forceinline__ void cp_async_wait_1() {
-    asm volatile("cp.async.wait_group 1;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -298,19 +261,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
           "=r"(r[31])
         : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-        "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
 
