@@ -215,8 +215,8 @@ def run_msa(args, rank, world, local_rank):
         clocks.start()
         time.sleep(0.3)
         t0.record()
-        for ev in evs:
-            step(ev)
+        for _ in range(steps):
+            step()
         t1.record()
         torch.cuda.synchronize()
         if world > 1:
@@ -226,6 +226,11 @@ def run_msa(args, rank, world, local_rank):
         st = msa.device_status(ws)
         if st != 0:
             raise RuntimeError(f"device status {msa.status_string(st)}")
+        # stage times from a second, separate pass (events between the stages
+        # would stop consecutive kernels from overlapping their launch)
+        for ev in evs:
+            step(ev)
+        torch.cuda.synchronize()
         stage_ms = {}
         for a, b in evs:
             for i, (s_, e_) in a.items():

@@ -14,15 +14,17 @@ namespace msa {
 // SIMT kernels (kernels_simt.cu)
 cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k_idx,
                                float *block_scores, int num_sms, cudaStream_t st);
+// pdl: allow programmatic dependent launch after the previous kernel in st
+// (the kernel waits for it before reading its results)
 cudaError_t launch_decode_select(const Shape &sh, const float *block_scores, int32_t *ids,
-                                 cudaStream_t st);
+                                 cudaStream_t st, bool pdl);
 size_t decode_attn_smem_bytes(const Shape &sh);
 cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, const void *v,
                                const int32_t *ids, float *part_o, float *part_lse, int S,
-                               int *status, cudaStream_t st);
+                               int *status, cudaStream_t st, bool pdl);
 cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            const float *part_lse, const int32_t *ids, float *out, float *lse,
-                           int S, cudaStream_t st);
+                           int S, cudaStream_t st, bool pdl);
 cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts,
                           int *pair_totals, int32_t *row_ptr, int32_t *entries, int *item_ptr,
                           AttnItem *items, int *counters, int rows_per_item, int n_chunks,

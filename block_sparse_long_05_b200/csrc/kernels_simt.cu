@@ -127,10 +127,19 @@ __global__ void __launch_bounds__(256) decode_index_scan_kernel(
 // bits); min(K, own+1)-1 rounds of block arg-max pick the winners (the owner
 // of a winner advances to its next best); own is added, ids written ascending.
 // ------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start before the previous kernel in its
+// stream has finished; this waits until that kernel has completed and its
+// writes are visible.  A no-op for kernels launched the ordinary way.
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 constexpr int kSelThreads = 1024;
 
 __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     const float *__restrict__ block_scores, int32_t *__restrict__ ids, int N, int own, int K) {
+    grid_dep_wait();  // inputs come from the previous kernel in the stream
     const int b = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     __shared__ uint64_t wbest[32];
@@ -235,6 +244,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ ids,
     float *__restrict__ part_o, float *__restrict__ part_lse, int T, int Hq, int Hkv, int block,
     int K, int S, int N, float scale_log2, int *__restrict__ status) {
+    grid_dep_wait();  // inputs come from the previous kernel in the stream
     constexpr int KS = kDecodeKeys;  // 64 keys = 4 warps x 16
     constexpr int STR = D + 8;       // padded row (bf16 elements)
     constexpr int PIECES = D / 8;    // 16-byte pieces per row
@@ -430,6 +440,7 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
     const PT *__restrict__ part_o, const float *__restrict__ part_lse,
     const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
     int K, int S, int HG, int G) {
+    grid_dep_wait();  // inputs come from the previous kernel in the stream
     constexpr int VEC = 16 / sizeof(PT);  // elements per 16-byte load
     constexpr int NV = D / VEC;           // 16-byte loads per head row
     extern __shared__ float wsm[];        // [P][HG] weights, then [HG] LSE
@@ -509,6 +520,7 @@ __global__ void __launch_bounds__(256) lse_combine_split_kernel(
     const PT *__restrict__ part_o, const float *__restrict__ part_lse,
     const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
     int K, int S) {
+    grid_dep_wait();  // inputs come from the previous kernel in the stream
     constexpr int PER = D / 32;  // elements per lane
     extern __shared__ float wsm[];                // [P] weights, then [8][D] sums
     const long long row = blockIdx.x;
@@ -774,6 +786,25 @@ __global__ void __launch_bounds__(256) attn_items_kernel(const int *__restrict__
 }  // namespace
 
 // ------------------------------------------------------------------ launchers
+// Launch `kernel`; with pdl the kernel may be scheduled while the previous
+// kernel in the stream drains (it calls grid_dep_wait before reading that
+// kernel's results), which hides the launch gap between dependent kernels.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k_idx,
                                float *block_scores, int num_sms, cudaStream_t st) {
     (void)num_sms;
@@ -807,10 +838,10 @@ cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k
 }
 
 cudaError_t launch_decode_select(const Shape &sh, const float *block_scores, int32_t *ids,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, bool pdl) {
     const int own = (sh.T - 1) / sh.block;
-    decode_select_kernel<<<sh.Bt, kSelThreads, 0, st>>>(block_scores, ids, sh.N, own, sh.K);
-    return cudaGetLastError();
+    return launch_ex(decode_select_kernel, dim3(sh.Bt), dim3(kSelThreads), 0, st, pdl, block_scores,
+                     ids, sh.N, own, sh.K);
 }
 
 size_t decode_attn_smem_bytes(const Shape &sh) {
@@ -820,7 +851,7 @@ size_t decode_attn_smem_bytes(const Shape &sh) {
 
 cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, const void *v,
                                const int32_t *ids, float *part_o, float *part_lse, int S,
-                               int *status, cudaStream_t st) {
+                               int *status, cudaStream_t st, bool pdl) {
     const long long grid = static_cast<long long>(sh.Bt) * sh.Hkv * sh.K * S;
     const size_t smem = decode_attn_smem_bytes(sh);
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(sh.d));
@@ -830,22 +861,22 @@ cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, co
     if (sh.d == 128) {
         cudaFuncSetAttribute(decode_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
-        decode_attn_kernel<128><<<static_cast<unsigned>(grid), 128, smem, st>>>(
-            qb, kb, vb, ids, part_o, part_lse, sh.T, sh.Hq, sh.Hkv, sh.block, sh.K, S, sh.N,
-            scale_log2, status);
+        return launch_ex(decode_attn_kernel<128>, dim3(static_cast<unsigned>(grid)), dim3(128), smem, st,
+                         pdl, qb, kb, vb, ids, part_o, part_lse, sh.T, sh.Hq, sh.Hkv, sh.block, sh.K,
+                         S, sh.N, scale_log2, status);
     } else {
         cudaFuncSetAttribute(decode_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
-        decode_attn_kernel<64><<<static_cast<unsigned>(grid), 128, smem, st>>>(
-            qb, kb, vb, ids, part_o, part_lse, sh.T, sh.Hq, sh.Hkv, sh.block, sh.K, S, sh.N,
-            scale_log2, status);
+        return launch_ex(decode_attn_kernel<64>, dim3(static_cast<unsigned>(grid)), dim3(128), smem, st,
+                         pdl, qb, kb, vb, ids, part_o, part_lse, sh.T, sh.Hq, sh.Hkv, sh.block, sh.K,
+                         S, sh.N, scale_log2, status);
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            const float *part_lse, const int32_t *ids, float *out, float *lse,
-                           int S, cudaStream_t st) {
+                           int S, cudaStream_t st, bool pdl) {
     const long long rows = static_cast<long long>(sh.Bt) * sh.n_q;
     if (rows * sh.Hq < 4096 && !part_bf16) {
         // few rows: split the partials of each (row, head) across 8 warps
@@ -856,13 +887,13 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
         if (sh.d == 128) {
             cudaFuncSetAttribute(lse_combine_split_kernel<float, 128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-            lse_combine_split_kernel<float, 128><<<grid, 256, smem, st>>>(po, part_lse, ids, out,
-                                                                         lse, sh.Hq, sh.K, S);
+            return launch_ex(lse_combine_split_kernel<float, 128>, grid, dim3(256), smem, st, pdl, po,
+                             part_lse, ids, out, lse, sh.Hq, sh.K, S);
         } else {
             cudaFuncSetAttribute(lse_combine_split_kernel<float, 64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-            lse_combine_split_kernel<float, 64><<<grid, 256, smem, st>>>(po, part_lse, ids, out,
-                                                                        lse, sh.Hq, sh.K, S);
+            return launch_ex(lse_combine_split_kernel<float, 64>, grid, dim3(256), smem, st, pdl, po,
+                             part_lse, ids, out, lse, sh.Hq, sh.K, S);
         }
         return cudaGetLastError();
     }
@@ -880,17 +911,18 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
     do {                                                                                         \
         cudaFuncSetAttribute(lse_combine_kernel<PT, DD>,                                         \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
-        lse_combine_kernel<PT, DD><<<grid, threads, smem, st>>>(                                 \
-            static_cast<const PT *>(part_o), part_lse, ids, out, lse, sh.Hq, sh.K, S, HG,        \
-            part_bf16 ? sh.G : 0);                                                               \
+        e = launch_ex(lse_combine_kernel<PT, DD>, grid, dim3(threads), smem, st, pdl,             \
+                      static_cast<const PT *>(part_o), part_lse, ids, out, lse, sh.Hq, sh.K, S,   \
+                      HG, part_bf16 ? sh.G : 0);                                                  \
     } while (0)
+    cudaError_t e = cudaSuccess;
     if (part_bf16) {
         if (sh.d == 128) MSA_COMBINE(__nv_bfloat16, 128); else MSA_COMBINE(__nv_bfloat16, 64);
     } else {
         if (sh.d == 128) MSA_COMBINE(float, 128); else MSA_COMBINE(float, 64);
     }
 #undef MSA_COMBINE
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts,

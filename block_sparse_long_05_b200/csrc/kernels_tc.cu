@@ -1410,7 +1410,7 @@ size_t prefill_attn_smem_bytes(const Shape &sh) {
 
 int prefill_attn_rows_per_item(int G) {
     const int tok = 128 / G;
-    return 32 * tok < kItemTokens ? 32 * tok : kItemTokens;
+    return 64 * tok < kItemTokens ? 64 * tok : kItemTokens;
 }
 
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,

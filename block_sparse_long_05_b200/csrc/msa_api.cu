@@ -189,7 +189,7 @@ msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids,
         if (launch_decode_scan(sh, q_idx, k_idx, scores, sms, st) != cudaSuccess) return MSA_ERR_CUDA;
         mark(ev, 0, false, st);
         mark(ev, 1, true, st);
-        if (launch_decode_select(sh, scores, ids, st) != cudaSuccess) return MSA_ERR_CUDA;
+        if (launch_decode_select(sh, scores, ids, st, true) != cudaSuccess) return MSA_ERR_CUDA;
         mark(ev, 1, false, st);
         return MSA_OK;
     }
@@ -250,11 +250,11 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
         float *po = at<float>(workspace, L.part_o);
         float *pl = at<float>(workspace, L.part_lse);
         mark(ev, 1, true, st);
-        cudaError_t e = launch_decode_attn(sh, q, k, v, ids, po, pl, S, status, st);
+        cudaError_t e = launch_decode_attn(sh, q, k, v, ids, po, pl, S, status, st, true);
         if (e != cudaSuccess) return MSA_ERR_CUDA;
         mark(ev, 1, false, st);
         mark(ev, 2, true, st);
-        e = launch_combine(sh, po, false, pl, ids, out, lse, S, st);
+        e = launch_combine(sh, po, false, pl, ids, out, lse, S, st, true);
         mark(ev, 2, false, st);
         return cuda_status(e);
     }
@@ -286,7 +286,7 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     mark(ev, 1, false, st);
     mark(ev, 2, true, st);
-    e = launch_combine(sh, po, true, pl, ids, out, lse, 1, st);
+    e = launch_combine(sh, po, true, pl, ids, out, lse, 1, st, true);
     mark(ev, 2, false, st);
     return cuda_status(e);
 }
