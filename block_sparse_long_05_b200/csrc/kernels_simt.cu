@@ -121,12 +121,6 @@ __global__ void __launch_bounds__(256) decode_index_scan_kernel(
     }
 }
 
-// ------------------------------------------------------------------------
-// Decode select: one CTA of 1024 threads per sequence.  Each thread keeps the
-// best of its strided candidates (key = score desc, block asc, packed in 64
-// bits); min(K, own+1)-1 rounds of block arg-max pick the winners (the owner
-// of a winner advances to its next best); own is added, ids written ascending.
-// ------------------------------------------------------------------------
 // Programmatic dependent launch: a kernel launched with the programmatic
 // stream-serialization attribute may start before the previous kernel in its
 // stream has finished; this waits until that kernel has completed and its
@@ -135,6 +129,13 @@ __device__ __forceinline__ void grid_dep_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// ------------------------------------------------------------------------
+// Decode select: one CTA of 1024 threads per sequence; a thread holds up to 8
+// strided candidates as 64-bit keys (score desc, block asc).  m =
+// min(K, own+1)-1 winners: every warp first extracts its own m best keys by
+// shuffles alone, then warp 0 merges the 32 sorted lists (m rounds of a warp
+// arg-max over the list heads).  own is added, ids written ascending.
+// ------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
 
 __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
     grid_dep_wait();  // inputs come from the previous kernel in the stream
     const int b = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __shared__ uint64_t wbest[32];
+    __shared__ uint64_t wtop[32 * kMaxK];  // per warp: its best keys, descending
     __shared__ int sel[kMaxK + 1];
     const float *sc = block_scores + static_cast<long long>(b) * N;
     const int m = min(K, own + 1) - 1;
@@ -155,6 +156,8 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
         mine[q] = j < own ? rank_key(sc[j], j) : 0;
         nm += j < own;
     }
+    // stage 1: every warp takes its own m best keys, in order, with shuffles
+    // only (keys are unique, so a winner has one owner)
     for (int p = 0; p < m; ++p) {
         uint64_t best = 0;
 #pragma unroll
@@ -164,25 +167,31 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
             const uint64_t other = shfl_xor_u64(best, o);
             best = other > best ? other : best;
         }
-        if (lane == 0) wbest[warp] = best;
-        __syncthreads();
-        if (warp == 0) {
-            uint64_t v = wbest[lane];
+        if (best != 0) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (mine[q] == best) mine[q] = 0;
+        }
+        if (lane == 0) wtop[warp * kMaxK + p] = best;  // 0: the warp has no more candidates
+    }
+    __syncthreads();
+    // stage 2: warp 0 merges the 32 descending lists, m rounds of a warp arg-max
+    // over the list heads; the winning list advances
+    if (warp == 0) {
+        int ptr = 0;
+        for (int p = 0; p < m; ++p) {
+            const uint64_t head = ptr < m ? wtop[lane * kMaxK + ptr] : 0;
+            uint64_t best = head;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
-                const uint64_t other = shfl_xor_u64(v, o);
-                v = other > v ? other : v;
+                const uint64_t other = shfl_xor_u64(best, o);
+                best = other > best ? other : best;
             }
-            if (lane == 0) wbest[0] = v;
+            if (head == best && best != 0) ++ptr;
+            if (lane == 0) sel[p] = 0x7FFFFFFF - static_cast<int>(static_cast<uint32_t>(best));
         }
-        __syncthreads();
-        const uint64_t win = wbest[0];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            if (mine[q] == win) mine[q] = 0;  // keys are unique: one owner
-        if (tid == 0) sel[p] = 0x7FFFFFFF - static_cast<int>(static_cast<uint32_t>(win));
-        __syncthreads();
     }
+    __syncthreads();
     (void)nm;
     if (tid == 0) {
         sel[m] = own;
