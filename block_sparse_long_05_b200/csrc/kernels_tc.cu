@@ -1398,8 +1398,6 @@ cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const
 size_t prefill_attn_smem_bytes(const Shape &sh) {
     const int NK = sh.block < 128 ? sh.block : 128;
     const int NS = sh.block / NK;
-    const int KVST = NS > 1 ? 2 : 1;
-    const int QBUF = NS > 1 ? 1 : 2;
     const size_t kv_tile = static_cast<size_t>(NK) * 128 * (sh.d / 64);
     const size_t q = static_cast<size_t>(sh.d / 64) * kRegionBytes + 2048;
     if (NS == 1)  // resident kernel: K/V, two Q tiles, two staging buffers, row statistics
