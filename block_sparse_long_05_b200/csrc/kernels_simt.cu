@@ -257,7 +257,6 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     constexpr int KS = kDecodeKeys;  // 64 keys = 4 warps x 16
     constexpr int STR = D + 8;       // padded row (bf16 elements)
     constexpr int PIECES = D / 8;    // 16-byte pieces per row
-    constexpr int NT = D / 8;        // n-tiles of the PV product
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __nv_bfloat16 *Ks = reinterpret_cast<__nv_bfloat16 *>(smem_raw);  // [KS][STR]
     __nv_bfloat16 *Vs = Ks + KS * STR;                                  // [KS][STR]
