@@ -162,6 +162,31 @@ def decode_bytes(w, ids):
     return scan, kv
 
 
+# ---------------------------------------------------------------- ranks
+def rank_seed(w, rank: int) -> int:
+    """Weak scaling: rank r runs its own Bt sequences of the workload, drawn
+    with seed w.seed + r (independent problems; no data-path collective)."""
+    return w.seed + rank
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise maximum of per-rank floats (step times) over all ranks;
+    every rank takes part and gets the result."""
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(w, ms: float, world: int) -> float:
+    """Whole-job tokens/s: the query tokens all ranks processed in one step
+    divided by the slowest rank's step time."""
+    return w.Bt * w.n_q * world / (ms / 1e3)
+
+
 # ---------------------------------------------------------------- MSA arm
 def run_msa(args, rank, world, local_rank):
     import torch
@@ -175,7 +200,7 @@ def run_msa(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
 
     def measure(w, steps, warmup, with_e2e):
-        x = make_inputs(w, device=dev, seed=w.seed + rank)
+        x = make_inputs(w, device=dev, seed=rank_seed(w, rank))
         ws = msa.Workspace.for_shape(w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K,
                                      device=dev)
         ids = torch.empty((w.Bt, w.n_q, w.K), dtype=torch.int32, device=dev)
@@ -237,10 +262,7 @@ def run_msa(args, rank, world, local_rank):
                 stage_ms[f"index{i}"] = stage_ms.get(f"index{i}", 0.0) + s_.elapsed_time(e_) / steps
             for i, (s_, e_) in b.items():
                 stage_ms[f"attn{i}"] = stage_ms.get(f"attn{i}", 0.0) + s_.elapsed_time(e_) / steps
-        if world > 1:
-            tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms = float(tt.item())
+        ms = max_over_ranks([ms], world, dev)[0]
         launches = (1 + 5 + 1 + 1) if not w.is_decode else \
             ((1 if (w.T - 1) // w.block > 0 else 0) + 1 + 1 + 1)
         res = {"ms": ms, "stage_ms": stage_ms, "clocks": clk, "launches": launches * steps}
@@ -320,10 +342,7 @@ def run_msa(args, rank, world, local_rank):
             ems = b0.elapsed_time(b1) / p_steps
             if msa.device_status(ws) != 0:
                 raise RuntimeError("device status after the pipelined e2e steps")
-            if world > 1:
-                tt = torch.tensor([ems, serial_ms], device=dev, dtype=torch.float64)
-                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-                ems, serial_ms = float(tt[0].item()), float(tt[1].item())
+            ems, serial_ms = max_over_ranks([ems, serial_ms], world, dev)
             res["e2e"] = {"ms": ems, "serial_ms": serial_ms, "h2d": h2d, "d2h": d2h,
                           "steps": p_steps}
             del sets
@@ -334,7 +353,7 @@ def run_msa(args, rank, world, local_rank):
 
     r = measure(w, args.steps, args.warmup, not args.no_e2e)
     tokens_per_step = w.Bt * w.n_q * world
-    value = tokens_per_step / (r["ms"] / 1e3)
+    value = job_throughput(w, r["ms"], world)
 
     # roofline of the dominant kernel
     sm = r["stage_ms"]
