@@ -1,5 +1,5 @@
 // ptx_sm100.cuh -- inline-PTX wrappers for sm_100a: mbarriers with bounded
-// waits, TMA tile loads (no cluster multicast), bulk copies, cache-policy
+// waits, TMA tile loads into this CTA only, bulk copies, cache-policy
 // loads, packed fp32 arithmetic, and the tcgen05 tensor-core / tensor-memory
 // instructions.
 //
