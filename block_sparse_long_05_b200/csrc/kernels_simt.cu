@@ -41,11 +41,13 @@ __device__ __forceinline__ uint64_t rank_key(float s, int j) {
     return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(0x7FFFFFFF - j);
 }
 
-__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
-    uint32_t lo = static_cast<uint32_t>(v), hi = static_cast<uint32_t>(v >> 32);
-    lo = __shfl_xor_sync(0xFFFFFFFFu, lo, m);
-    hi = __shfl_xor_sync(0xFFFFFFFFu, hi, m);
-    return (static_cast<uint64_t>(hi) << 32) | lo;
+// Warp-wide maximum of 64-bit keys in two reductions: the largest high word,
+// then the largest low word among the lanes that hold it.
+__device__ __forceinline__ uint64_t warp_max_key(uint64_t key) {
+    const uint32_t hi = static_cast<uint32_t>(key >> 32), lo = static_cast<uint32_t>(key);
+    const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+    const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+    return (static_cast<uint64_t>(mhi) << 32) | mlo;
 }
 
 // ------------------------------------------------------------------------
@@ -132,9 +134,10 @@ __device__ __forceinline__ void grid_dep_wait() {
 // ------------------------------------------------------------------------
 // Decode select: one CTA of 1024 threads per sequence; a thread holds up to 8
 // strided candidates as 64-bit keys (score desc, block asc).  m =
-// min(K, own+1)-1 winners: every warp first extracts its own m best keys by
-// shuffles alone, then warp 0 merges the 32 sorted lists (m rounds of a warp
-// arg-max over the list heads).  own is added, ids written ascending.
+// min(K, own+1)-1 winners: every warp first extracts its own m best keys with
+// warp max-reductions (redux.sync on the high, then the low word), then warp 0
+// merges the 32 sorted lists (m rounds of a warp arg-max over the list
+// heads).  own is added; each id is written at its rank (ascending).
 // ------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
 
@@ -156,17 +159,13 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
         mine[q] = j < own ? rank_key(sc[j], j) : 0;
         nm += j < own;
     }
-    // stage 1: every warp takes its own m best keys, in order, with shuffles
-    // only (keys are unique, so a winner has one owner)
+    // stage 1: every warp takes its own m best keys, in order, with warp
+    // reductions only (keys are unique, so a winner has one owner)
     for (int p = 0; p < m; ++p) {
         uint64_t best = 0;
 #pragma unroll
         for (int q = 0; q < 8; ++q) best = mine[q] > best ? mine[q] : best;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const uint64_t other = shfl_xor_u64(best, o);
-            best = other > best ? other : best;
-        }
+        best = warp_max_key(best);
         if (best != 0) {
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -181,31 +180,25 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(
         int ptr = 0;
         for (int p = 0; p < m; ++p) {
             const uint64_t head = ptr < m ? wtop[lane * kMaxK + ptr] : 0;
-            uint64_t best = head;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const uint64_t other = shfl_xor_u64(best, o);
-                best = other > best ? other : best;
-            }
+            const uint64_t best = warp_max_key(head);
             if (head == best && best != 0) ++ptr;
             if (lane == 0) sel[p] = 0x7FFFFFFF - static_cast<int>(static_cast<uint32_t>(best));
         }
+        if (lane == 0) sel[m] = own;
     }
     __syncthreads();
     (void)nm;
-    if (tid == 0) {
-        sel[m] = own;
-        const int n = m + 1;
-        for (int a = 1; a < n; ++a) {  // insertion sort, ascending
-            const int x = sel[a];
-            int c = a - 1;
-            while (c >= 0 && sel[c] > x) {
-                sel[c + 1] = sel[c];
-                --c;
-            }
-            sel[c + 1] = x;
+    // ids ascending: each of the n = m + 1 distinct winners is written at its
+    // rank; the slots after them get -1
+    const int n = m + 1;
+    if (tid < K) {
+        int v = -1, slot = tid;
+        if (tid < n) {
+            v = sel[tid];
+            slot = 0;
+            for (int c = 0; c < n; ++c) slot += sel[c] < v;
         }
-        for (int s = 0; s < K; ++s) ids[static_cast<long long>(b) * K + s] = s < n ? sel[s] : -1;
+        ids[static_cast<long long>(b) * K + slot] = v;
     }
 }
 
@@ -520,17 +513,21 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
     }
 }
 
-// Few query rows (decode): one CTA of 8 warps per (row, head); warp w merges
-// partials p = w, w+8, ... of that head and the warps' sums are added in
-// shared memory.  Same arithmetic as lse_combine_kernel.
+// Few query rows (decode): one CTA of kCombineSplitWarps warps per (row,
+// head) -- small CTAs, so that the grid fits the GPU in one wave; warp w
+// merges partials p = w, w+NW, ... of that head and the warps' sums are added
+// in shared memory.  Same arithmetic as lse_combine_kernel.
+constexpr int kCombineSplitWarps = 4;
+
 template <typename PT, int D>
-__global__ void __launch_bounds__(256) lse_combine_split_kernel(
+__global__ void __launch_bounds__(32 * kCombineSplitWarps) lse_combine_split_kernel(
     const PT *__restrict__ part_o, const float *__restrict__ part_lse,
     const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
     int K, int S) {
     grid_dep_wait();  // inputs come from the previous kernel in the stream
     constexpr int PER = D / 32;  // elements per lane
-    extern __shared__ float wsm[];                // [P] weights, then [8][D] sums
+    constexpr int NW = kCombineSplitWarps;
+    extern __shared__ float wsm[];                // [P] weights, then [NW][D] sums
     const long long row = blockIdx.x;
     const int h = blockIdx.y;
     const int P = K * S;
@@ -571,7 +568,7 @@ __global__ void __launch_bounds__(256) lse_combine_split_kernel(
     const long long pstride = static_cast<long long>(Hq) * D;
     const PT *src = part_o + (row * K * S * Hq + h) * static_cast<long long>(D) + lane * PER;
 #pragma unroll 4
-    for (int pp = warp; pp < P; pp += 8) {
+    for (int pp = warp; pp < P; pp += NW) {
         const float wgt = wsm[pp];
         const PT *sp = src + pp * pstride;
         float f[PER];
@@ -591,7 +588,7 @@ __global__ void __launch_bounds__(256) lse_combine_split_kernel(
     for (int c = tid; c < D; c += blockDim.x) {
         float a = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) a += acc_s[w * D + c];
+        for (int w = 0; w < NW; ++w) a += acc_s[w * D + c];
         out[(row * Hq + h) * static_cast<long long>(D) + c] = a;
     }
     if (tid == 0) lse_out[row * Hq + h] = L_s;
@@ -887,20 +884,22 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            int S, cudaStream_t st, bool pdl) {
     const long long rows = static_cast<long long>(sh.Bt) * sh.n_q;
     if (rows * sh.Hq < 4096 && !part_bf16) {
-        // few rows: split the partials of each (row, head) across 8 warps
+        // few rows: split the partials of each (row, head) across the warps of a CTA
         const int P = sh.K * S;
-        const size_t smem = (static_cast<size_t>((P + 3) & ~3) + 8 * sh.d) * sizeof(float);
+        const size_t smem =
+            (static_cast<size_t>((P + 3) & ~3) + static_cast<size_t>(kCombineSplitWarps) * sh.d) *
+            sizeof(float);
         const dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>(sh.Hq));
         const auto *po = static_cast<const float *>(part_o);
         if (sh.d == 128) {
             cudaFuncSetAttribute(lse_combine_split_kernel<float, 128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-            return launch_ex(lse_combine_split_kernel<float, 128>, grid, dim3(256), smem, st, pdl, po,
+            return launch_ex(lse_combine_split_kernel<float, 128>, grid, dim3(32 * kCombineSplitWarps), smem, st, pdl, po,
                              part_lse, ids, out, lse, sh.Hq, sh.K, S);
         } else {
             cudaFuncSetAttribute(lse_combine_split_kernel<float, 64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-            return launch_ex(lse_combine_split_kernel<float, 64>, grid, dim3(256), smem, st, pdl, po,
+            return launch_ex(lse_combine_split_kernel<float, 64>, grid, dim3(32 * kCombineSplitWarps), smem, st, pdl, po,
                              part_lse, ids, out, lse, sh.Hq, sh.K, S);
         }
         return cudaGetLastError();
