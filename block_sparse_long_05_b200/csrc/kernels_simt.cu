@@ -513,20 +513,18 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
     }
 }
 
-// Few query rows (decode): one CTA of kCombineSplitWarps warps per (row,
-// head) -- small CTAs, so that the grid fits the GPU in one wave; warp w
+// Few query rows (decode): one CTA of NW warps per (row, head); warp w
 // merges partials p = w, w+NW, ... of that head and the warps' sums are added
-// in shared memory.  Same arithmetic as lse_combine_kernel.
-constexpr int kCombineSplitWarps = 4;
-
-template <typename PT, int D>
-__global__ void __launch_bounds__(32 * kCombineSplitWarps) lse_combine_split_kernel(
+// in shared memory.  Same arithmetic as lse_combine_kernel.  NW = 8 while the
+// grid fits the GPU in one wave of 8-warp CTAs, else 4 (smaller CTAs: one
+// wave for twice the grid).
+template <typename PT, int D, int NW>
+__global__ void __launch_bounds__(32 * NW) lse_combine_split_kernel(
     const PT *__restrict__ part_o, const float *__restrict__ part_lse,
     const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
     int K, int S) {
     grid_dep_wait();  // inputs come from the previous kernel in the stream
     constexpr int PER = D / 32;  // elements per lane
-    constexpr int NW = kCombineSplitWarps;
     extern __shared__ float wsm[];                // [P] weights, then [NW][D] sums
     const long long row = blockIdx.x;
     const int h = blockIdx.y;
@@ -885,24 +883,30 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
     const long long rows = static_cast<long long>(sh.Bt) * sh.n_q;
     if (rows * sh.Hq < 4096 && !part_bf16) {
         // few rows: split the partials of each (row, head) across the warps of a CTA
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const bool wide = rows * sh.Hq <= static_cast<long long>(sms) * 8;  // one wave of 8-warp CTAs
+        const int nw = wide ? 8 : 4;
         const int P = sh.K * S;
-        const size_t smem =
-            (static_cast<size_t>((P + 3) & ~3) + static_cast<size_t>(kCombineSplitWarps) * sh.d) *
-            sizeof(float);
+        const size_t smem = (static_cast<size_t>((P + 3) & ~3) + static_cast<size_t>(nw) * sh.d) *
+                            sizeof(float);
         const dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>(sh.Hq));
         const auto *po = static_cast<const float *>(part_o);
+#define MSA_COMBINE_SPLIT(DD, NWW)                                                                \
+    do {                                                                                          \
+        cudaFuncSetAttribute(lse_combine_split_kernel<float, DD, NWW>,                            \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
+        return launch_ex(lse_combine_split_kernel<float, DD, NWW>, grid, dim3(32 * NWW), smem, st, \
+                         pdl, po, part_lse, ids, out, lse, sh.Hq, sh.K, S);                        \
+    } while (0)
         if (sh.d == 128) {
-            cudaFuncSetAttribute(lse_combine_split_kernel<float, 128>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-            return launch_ex(lse_combine_split_kernel<float, 128>, grid, dim3(32 * kCombineSplitWarps), smem, st, pdl, po,
-                             part_lse, ids, out, lse, sh.Hq, sh.K, S);
-        } else {
-            cudaFuncSetAttribute(lse_combine_split_kernel<float, 64>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-            return launch_ex(lse_combine_split_kernel<float, 64>, grid, dim3(32 * kCombineSplitWarps), smem, st, pdl, po,
-                             part_lse, ids, out, lse, sh.Hq, sh.K, S);
+            if (wide) MSA_COMBINE_SPLIT(128, 8);
+            MSA_COMBINE_SPLIT(128, 4);
         }
-        return cudaGetLastError();
+        if (wide) MSA_COMBINE_SPLIT(64, 8);
+        MSA_COMBINE_SPLIT(64, 4);
+#undef MSA_COMBINE_SPLIT
     }
     // heads per CTA: all of them when there are many rows, else fewer so the
     // grid still covers the SMs a few times
