@@ -175,6 +175,35 @@ def check_index_bruteforce(o):
         assert np.array_equal(got_r, exp[rows])
 
 
+def check_index_scores_bruteforce(o):
+    """s(t, j) equals the maximum of the exact integer dot products over the
+    keys of block j (NaN for j >= own(t)), including blocks whose products
+    are all negative."""
+    cases = [(Bt, n_q, T, block, d_idx, 200 + n, None)
+             for n, (Bt, n_q, T, block, _, d_idx) in enumerate(INDEX_SHAPES)]
+    cases.append((1, 20, 20, 4, 3, 0, "negative"))  # every product is -3
+    for Bt, n_q, T, block, d_idx, seed, kind in cases:
+        if kind == "negative":
+            qi = bf16(np.ones((Bt, n_q, d_idx)))
+            ki = bf16(-np.ones((Bt, T, d_idx)))
+        else:
+            _, _, _, qi, ki = rand_case(Bt, n_q, T, 1, 1, 1, d_idx, seed=seed)
+        sc = o.index_scores(qi, ki, Bt, n_q, T, d_idx, block)
+        Q = qi.float().numpy().astype(np.int64)
+        Kk = ki.float().numpy().astype(np.int64)
+        for b in range(Bt):
+            S = Q[b] @ Kk[b].T
+            for i in range(n_q):
+                t = T - n_q + i
+                own = t // block
+                row = sc[b * n_q + i]
+                for j in range((T + block - 1) // block):
+                    if j < own:
+                        assert row[j] == S[i, j * block:(j + 1) * block].max(), (b, i, j)
+                    else:
+                        assert np.isnan(row[j]), (b, i, j)
+
+
 def check_index_invariants(o):
     Bt, n_q, T, block, K, d_idx = 2, 200, 200, 8, 5, 6
     _, _, _, qi, ki = rand_case(Bt, n_q, T, 1, 1, 1, d_idx, seed=7)
@@ -326,6 +355,7 @@ ALL_CHECKS = [
     check_index_golden,
     check_attention_golden,
     check_index_bruteforce,
+    check_index_scores_bruteforce,
     check_index_invariants,
     check_index_ties,
     check_attention_sdpa_sparse,

@@ -21,6 +21,13 @@ MUTANTS = [
     ("index_scores_negated", "dot += bf16_bits_to_double(q_idx_row[c]) * bf16_bits_to_double(krow[c]);",
      "dot -= bf16_bits_to_double(q_idx_row[c]) * bf16_bits_to_double(krow[c]);", 1),
     ("combine_weight_sign", "double w = exp(l - L);", "double w = exp(L - l);", 1),
+    ("query_position_from_sequence_start", "*t = (int64_t)T - n_q + (r % n_q);",
+     "*t = (r % n_q);", 1),
+    ("index_max_starts_at_zero", "double best = -INFINITY;", "double best = 0.0;", 1),
+    ("own_block_one_late", "int own = (int)(t / block);", "int own = (int)((t + 1) / block);", 2),
+    ("own_block_not_forced", "sel[n_sel++] = own;", "(void)own;", 1),
+    ("softmax_not_normalised", "double p = exp(x[n++] - l);", "double p = exp(x[n++] - mx);", 1),
+    ("combine_lse_drops_max", "double L = mx + log(sum);", "double L = log(sum);", 1),
     ("invert_unsorted", "for (int i = 0; i < n_q; ++i)\n            for (int s = 0; s < K; ++s) {\n                int64_t r",
      "for (int i = n_q - 1; i >= 0; --i)\n            for (int s = 0; s < K; ++s) {\n                int64_t r", 1),
 ]
