@@ -37,6 +37,7 @@ def _decode_case(w, index_values="int3"):
     Workload("dec_dense", 2, 1, 700, 8, 1, 64, 128, 16, 64),         # K >= N, G = 8
     Workload("dec_k1", 2, 1, 3000, 8, 2, 128, 512, 1, 128),          # own block only
     Workload("dec_k32", 1, 1, 20000, 4, 1, 64, 32, 32, 64),          # K = 32, block 32
+    Workload("dec_max_blocks", 2, 1, 8192 * 32, 4, 1, 64, 32, 32, 64),  # N = 8192: 8 per select thread
 ], ids=lambda w: w.name)
 def test_decode_small(w):
     _decode_case(w)

@@ -143,6 +143,13 @@ def test_attention_score_spread(w, rising):
     _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)
 
 
+def test_prefill_max_blocks():
+    # N = 8192 blocks (the largest supported: inversion histograms of 4 x N
+    # counters in shared memory) and K = 32 (the largest): the last 256
+    # queries of a 262144-key context with 32-key blocks, every row checked
+    _end_to_end(Workload("pf_max_blocks", 1, 256, 8192 * 32, 4, 1, 64, 32, 32, 64))
+
+
 @pytest.mark.parametrize("w", [PREFILL_64K, PREFILL_256K], ids=lambda w: w.name)
 def test_prefill_full_size_sampled(w):
     _end_to_end(w, rows=sample_rows(w, N_SAMPLE))
