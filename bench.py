@@ -432,6 +432,25 @@ def run_msa(args, rank, world, local_rank):
             "scan_frac": scan_b / (smd["index0"] / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
         }
 
+    # decode step at this prefill workload's context: one sequence of T keys,
+    # same heads, block, K and index dim (a failure here is reported in the
+    # object and leaves the line above intact)
+    if not args.no_decode and not w.is_decode and world == 1:
+        from block_sparse_long_05_b200.inputs import Workload
+        wt = Workload(f"decode_1x{w.T}", 1, 1, w.T, w.Hq, w.Hkv, w.d, w.block, w.K, w.d_idx)
+        try:
+            rt = measure(wt, max(args.steps, 20), max(args.warmup, 3), False)
+            scan_b, kv_b = decode_bytes(wt, rt["ids"])
+            line["decode_at_T"] = {
+                "workload": wt.name, "value": 1 / (rt["ms"] / 1e3), "unit": UNIT,
+                "ms_per_step": rt["ms"],
+                "stage_ms": {k: round(v, 4) for k, v in rt["stage_ms"].items()},
+                "step_bytes": scan_b + kv_b,
+                "step_hbm_frac": (scan_b + kv_b) / (rt["ms"] / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
+            }
+        except Exception as e:  # noqa: BLE001 -- recorded, not hidden
+            line["decode_at_T"] = {"workload": wt.name, "error": f"{type(e).__name__}: {e}"[:300]}
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     return line
