@@ -5,4 +5,5 @@ Python binding, ``inputs`` the seeded synthetic workloads, ``build`` the nvcc
 build of the library.
 """
 from .msa import (MSAError, Workspace, device_status, index_topk, load_library,  # noqa: F401
-                  select_invert, selftest_umma, sparse_attn, status_string, workspace_size)
+                  select_invert, selftest_umma, sparse_attn, sparse_attn_decode_noalloc,
+                  status_string, workspace_size)
