@@ -38,6 +38,7 @@ def _decode_case(w, index_values="int3"):
     Workload("dec_k1", 2, 1, 3000, 8, 2, 128, 512, 1, 128),          # own block only
     Workload("dec_k32", 1, 1, 20000, 4, 1, 64, 32, 32, 64),          # K = 32, block 32
     Workload("dec_max_blocks", 2, 1, 8192 * 32, 4, 1, 64, 32, 32, 64),  # N = 8192: 8 per select thread
+    Workload("dec_many_heads", 48, 1, 3000, 32, 4, 64, 64, 4, 64),   # 4-warp split combine at d = 64
 ], ids=lambda w: w.name)
 def test_decode_small(w):
     _decode_case(w)
