@@ -54,3 +54,35 @@ def test_decode_bytes():
     keys = (32 + 32 + 4) + (32 + 4)  # block 3 holds keys 96..99
     assert kv == keys * w.Hkv * w.d * 2 * 2 + w.Bt * w.Hq * w.d * 2
     assert np.isclose(bench.job_throughput(w, 0.5, 4), 2 * 1 * 4 / 0.5e-3)
+
+
+def _host_run(mode):
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "tests", "bench_host_worker.py"), mode],
+                       cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    return json.loads(r.stdout.strip().splitlines()[-1])
+
+
+def test_bench_line_structure_with_and_without_l2_flush():
+    """bench.py's measurement logic end to end on the CPU (library, events and
+    clocks faked): the JSON line carries every key the benchmark contract
+    names, for both timing paths, with both decode secondaries."""
+    for mode, l2_word in (("flush", "flushed"), ("noflush", "no flush")):
+        line = _host_run(mode)
+        for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                    "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                    "gpu_launches", "roofline", "clocks", "decode", "decode_at_T"):
+            assert key in line, (mode, key)
+        assert l2_word in line["config"]["l2"], (mode, line["config"]["l2"])
+        assert line["gpu_launches"] == 8 * line["steps"]
+        for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+            assert key in line["roofline"], key
+        assert "error" not in line["decode_at_T"], line["decode_at_T"]
+        assert line["decode_at_T"]["workload"] == f"decode_1x{line['config']['T']}"
+        if mode == "flush":  # fake events tick 0.25 ms per record: one step = 0.25 ms
+            assert abs(line["ms_per_step"] - 0.25) < 1e-9
