@@ -162,9 +162,10 @@ __global__ void __launch_bounds__(128, 1) selftest_umma_kernel(
 
 // ===========================================================================
 // Prefill index kernel.
-//   warp 0: TMA producer (q tile once per item, 128-key k tiles through a
-//           4-stage ring), warp 1: MMA issuer (TMEM owner), warps 2-5:
-//           epilogue (row = 32*(warp%4) + lane; block max-pool + top-K).
+//   warp 0: TMA producer (q tile once per item, kIdxKeys-key k tiles through
+//           a kIdxStages-stage ring), warp 1: MMA issuer (TMEM owner: two
+//           accumulators of kIdxKeys columns), warps 2-5: epilogue
+//           (row = 32*(warp%4) + lane; block max-pool + top-K).
 // Work item = (sequence b, 128-query tile qt); items ordered by decreasing
 // cost and dealt to CTAs in a snake order.
 // ===========================================================================
