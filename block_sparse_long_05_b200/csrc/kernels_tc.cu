@@ -438,13 +438,14 @@ struct ItemRows {
 // Prefill attention, K/V block resident (block <= 128): warp-specialised.
 //   warps 0-3 / 4-7: softmax warpgroups SG0 / SG1.  Each takes alternate
 //     128-row chunks of the item: wait for S (which releases the Q tile),
-//     softmax (S -> P in tensor memory), hand the row statistics to the
-//     epilogue warpgroup, issue PV, wait for it, issue S of its next chunk.
-//     One elected thread per warpgroup issues that warpgroup's tcgen05.mma.
+//     softmax (S -> P in tensor memory), store the rows' lse, hand 1/l to
+//     the epilogue warpgroup, issue PV, wait for it, issue S of its next
+//     chunk.  One elected thread per warpgroup issues that warpgroup's
+//     tcgen05.mma.
 //   warps 8-11: epilogue warpgroup.  For every chunk in order: read O from
-//     tensor memory (which frees it for the next PV), normalise, stage the
-//     bf16 partial rows token-major in one of two staging buffers and write
-//     each token's G rows with one bulk copy; store lse.
+//     tensor memory (which frees it for the next PV), scale by 1/l, stage
+//     the bf16 partial rows token-major in one of two staging buffers and
+//     write each token's G rows with one bulk copy.
 //   warps 12-15: producers.  Thread 0 of them TMA-loads K_j and V_j once per
 //     item; all gather the Q rows of chunks 0, 1, 2, ... into the owning
 //     softmax warpgroup's Q tile: rows are loaded into registers (not
