@@ -12,8 +12,11 @@
 namespace msa {
 
 // SIMT kernels (kernels_simt.cu)
+// pm: paged k_idx / K / V (pm.table == nullptr: contiguous); bad page ids
+// are skipped and reported in *status
 cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k_idx,
-                               float *block_scores, int num_sms, cudaStream_t st);
+                               float *block_scores, const PageMap &pm, int *status, int num_sms,
+                               cudaStream_t st);
 // pdl: allow programmatic dependent launch after the previous kernel in st
 // (the kernel waits for it before reading its results)
 cudaError_t launch_decode_select(const Shape &sh, const float *block_scores, int32_t *ids,
@@ -21,7 +24,7 @@ cudaError_t launch_decode_select(const Shape &sh, const float *block_scores, int
 size_t decode_attn_smem_bytes(const Shape &sh);
 cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, const void *v,
                                const int32_t *ids, float *part_o, float *part_lse, int S,
-                               int *status, cudaStream_t st, bool pdl);
+                               const PageMap &pm, int *status, cudaStream_t st, bool pdl);
 cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            const float *part_lse, const int32_t *ids, float *out, float *lse,
                            int S, cudaStream_t st, bool pdl);

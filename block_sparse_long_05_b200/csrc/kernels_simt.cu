@@ -67,7 +67,8 @@ __device__ __forceinline__ uint4 ld_stream16(const uint4 *p) {
 template <int D_IDX>
 __global__ void __launch_bounds__(256) decode_index_scan_kernel(
     const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16 *__restrict__ k_idx,
-    float *__restrict__ block_scores, int Bt, int T, int block, int own, int N, int rw, int bpc) {
+    float *__restrict__ block_scores, int Bt, int T, int block, int own, int N, int rw, int bpc,
+    PageMap pm, int *__restrict__ status) {
     // rw: rows per warp (a warp's rows lie in one block); bpc: blocks per CTA
     constexpr int LPR = D_IDX / 8;  // lanes per key row
     constexpr int RPL = 32 / LPR;   // key rows per warp load
@@ -77,16 +78,29 @@ __global__ void __launch_bounds__(256) decode_index_scan_kernel(
     const int sub = lane / LPR, part = lane % LPR;
     const int wpb = 8 / bpc;                         // warps per block
     const long long item = static_cast<long long>(blockIdx.x) * bpc + warp / wpb;
-    const bool active = item < static_cast<long long>(Bt) * own;
+    bool active = item < static_cast<long long>(Bt) * own;
     float best = -FLT_MAX;
+    long long row0 = 0;  // first k_idx row of the block in the (paged or contiguous) store
     if (active) {
         const int b = static_cast<int>(item / own), j = static_cast<int>(item % own);
+        if (pm.table) {
+            const int phys = pm.table[static_cast<long long>(b) * pm.stride + j];
+            if (phys < 0 || phys >= pm.count) {  // skipped (scores -FLT_MAX) and reported
+                active = false;
+                if (lane == 0 && warp % (8 / bpc) == 0) atomicOr(status, kDevBadIds);
+            }
+            row0 = static_cast<long long>(phys) * block;
+        } else {
+            row0 = static_cast<long long>(b) * T + static_cast<long long>(j) * block;
+        }
+    }
+    if (active) {
+        const int b = static_cast<int>(item / own);
         float qv[8];
         bf16x8_to_f32(*reinterpret_cast<const uint4 *>(q_idx + static_cast<long long>(b) * D_IDX + part * 8), qv);
         // the wpb warps of block j interleave over its row groups
         const int wi = warp % wpb;
-        const uint4 *base = reinterpret_cast<const uint4 *>(
-            k_idx + (static_cast<long long>(b) * T + static_cast<long long>(j) * block) * D_IDX);
+        const uint4 *base = reinterpret_cast<const uint4 *>(k_idx + row0 * D_IDX);
         const int groups = rw / RPL;  // row groups per warp
         for (int g0 = 0; g0 < groups; g0 += UNR) {
             uint4 ku[UNR];
@@ -245,7 +259,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
     const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ ids,
     float *__restrict__ part_o, float *__restrict__ part_lse, int T, int Hq, int Hkv, int block,
-    int K, int S, int N, float scale_log2, int *__restrict__ status) {
+    int K, int S, int N, float scale_log2, PageMap pm, int *__restrict__ status) {
     grid_dep_wait();  // inputs come from the previous kernel in the stream
     constexpr int KS = kDecodeKeys;  // 64 keys = 4 warps x 16
     constexpr int STR = D + 8;       // padded row (bf16 elements)
@@ -272,7 +286,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     const int t = T - 1;
     const int j = ids[static_cast<long long>(b) * K + s];
     int nk = 0;
-    long long k0 = 0;
+    long long k0 = 0, row0 = 0;  // first key (logical position) and its row in the store
     if (j >= N || j < -1) {
         if (tid == 0) atomicOr(status, kDevBadIds);
     } else if (j >= 0) {
@@ -283,14 +297,24 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
         if (k1 > T) k1 = T;
         if (k1 > t + 1) k1 = t + 1;
         nk = k1 > k0 ? static_cast<int>(k1 - k0) : 0;
+        if (pm.table) {
+            const int phys = pm.table[static_cast<long long>(b) * pm.stride + j];
+            if (phys < 0 || phys >= pm.count) {  // skipped and reported
+                if (tid == 0) atomicOr(status, kDevBadIds);
+                nk = 0;
+            }
+            row0 = static_cast<long long>(phys) * block + static_cast<long long>(sp) * KS;
+        } else {
+            row0 = static_cast<long long>(b) * T + k0;
+        }
     }
     if (nk == 0) {
         for (int g = tid; g < G; g += blockDim.x) part_lse[prow * Hq + hk * G + g] = -INFINITY;
         return;
     }
     // stage K and V rows (zero past nk)
-    const __nv_bfloat16 *kbase = k + ((static_cast<long long>(b) * T + k0) * Hkv + hk) * D;
-    const __nv_bfloat16 *vbase = v + ((static_cast<long long>(b) * T + k0) * Hkv + hk) * D;
+    const __nv_bfloat16 *kbase = k + (row0 * Hkv + hk) * D;
+    const __nv_bfloat16 *vbase = v + (row0 * Hkv + hk) * D;
     for (int e = tid; e < KS * PIECES; e += blockDim.x) {
         const int r = e / PIECES, c = e % PIECES;
         const bool ok = r < nk;
@@ -809,7 +833,8 @@ static cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 }
 
 cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k_idx,
-                               float *block_scores, int num_sms, cudaStream_t st) {
+                               float *block_scores, const PageMap &pm, int *status, int num_sms,
+                               cudaStream_t st) {
     (void)num_sms;
     const int own = (sh.T - 1) / sh.block;
     if (own > 0) {
@@ -832,10 +857,10 @@ cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k
         const auto *ki = static_cast<const __nv_bfloat16 *>(k_idx);
         if (sh.d_idx == 128)
             decode_index_scan_kernel<128><<<static_cast<unsigned>(grid), 256, 0, st>>>(
-                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N, rw, bpc);
+                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N, rw, bpc, pm, status);
         else
             decode_index_scan_kernel<64><<<static_cast<unsigned>(grid), 256, 0, st>>>(
-                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N, rw, bpc);
+                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N, rw, bpc, pm, status);
     }
     return cudaGetLastError();
 }
@@ -854,7 +879,7 @@ size_t decode_attn_smem_bytes(const Shape &sh) {
 
 cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, const void *v,
                                const int32_t *ids, float *part_o, float *part_lse, int S,
-                               int *status, cudaStream_t st, bool pdl) {
+                               const PageMap &pm, int *status, cudaStream_t st, bool pdl) {
     const long long grid = static_cast<long long>(sh.Bt) * sh.Hkv * sh.K * S;
     const size_t smem = decode_attn_smem_bytes(sh);
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(sh.d));
@@ -866,13 +891,13 @@ cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, co
                              static_cast<int>(smem));
         return launch_ex(decode_attn_kernel<128>, dim3(static_cast<unsigned>(grid)), dim3(128), smem, st,
                          pdl, qb, kb, vb, ids, part_o, part_lse, sh.T, sh.Hq, sh.Hkv, sh.block, sh.K,
-                         S, sh.N, scale_log2, status);
+                         S, sh.N, scale_log2, pm, status);
     } else {
         cudaFuncSetAttribute(decode_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
         return launch_ex(decode_attn_kernel<64>, dim3(static_cast<unsigned>(grid)), dim3(128), smem, st,
                          pdl, qb, kb, vb, ids, part_o, part_lse, sh.T, sh.Hq, sh.Hkv, sh.block, sh.K,
-                         S, sh.N, scale_log2, status);
+                         S, sh.N, scale_log2, pm, status);
     }
     return cudaGetLastError();
 }

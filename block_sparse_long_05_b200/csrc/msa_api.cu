@@ -186,7 +186,8 @@ msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids,
     if (n_q == 1) {
         float *scores = at<float>(workspace, L.block_scores);
         mark(ev, 0, true, st);
-        if (launch_decode_scan(sh, q_idx, k_idx, scores, sms, st) != cudaSuccess) return MSA_ERR_CUDA;
+        if (launch_decode_scan(sh, q_idx, k_idx, scores, PageMap{}, status, sms, st) != cudaSuccess)
+            return MSA_ERR_CUDA;
         mark(ev, 0, false, st);
         mark(ev, 1, true, st);
         if (launch_decode_select(sh, scores, ids, st, true) != cudaSuccess) return MSA_ERR_CUDA;
@@ -250,7 +251,7 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
         float *po = at<float>(workspace, L.part_o);
         float *pl = at<float>(workspace, L.part_lse);
         mark(ev, 1, true, st);
-        cudaError_t e = launch_decode_attn(sh, q, k, v, ids, po, pl, S, status, st, true);
+        cudaError_t e = launch_decode_attn(sh, q, k, v, ids, po, pl, S, PageMap{}, status, st, true);
         if (e != cudaSuccess) return MSA_ERR_CUDA;
         mark(ev, 1, false, st);
         mark(ev, 2, true, st);
@@ -289,6 +290,57 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     e = launch_combine(sh, po, true, pl, ids, out, lse, 1, st, true);
     mark(ev, 2, false, st);
     return cuda_status(e);
+}
+
+msa_status msa_index_topk_paged(const void *q_idx, const void *k_idx_pages,
+                                const int32_t *page_table, int page_stride, int num_pages,
+                                int32_t *ids, int Bt, int T, int d_idx, int block, int K,
+                                void *workspace, size_t workspace_bytes, void *stream) {
+    if (!q_idx || !k_idx_pages || !page_table || !ids) return MSA_ERR_INVALID_ARG;
+    Shape sh;
+    msa_status s = validate(Bt, 1, T, 1, 1, 64, d_idx, block, K, true, false, &sh);
+    if (s != MSA_OK) return s;
+    if (page_stride < sh.N || num_pages < 1) return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx_pages) || (reinterpret_cast<uintptr_t>(page_table) & 3))
+        return MSA_ERR_INVALID_ARG;
+    const WsLayout L = layout_for(sh, false);
+    if ((s = check_ws(workspace, workspace_bytes, L)) != MSA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int sms = num_sms_current();
+    if (sms <= 0) return MSA_ERR_CUDA;
+    int *status = at<int>(workspace, L.status);
+    float *scores = at<float>(workspace, L.block_scores);
+    const PageMap pm{page_table, page_stride, num_pages};
+    if (launch_decode_scan(sh, q_idx, k_idx_pages, scores, pm, status, sms, st) != cudaSuccess)
+        return MSA_ERR_CUDA;
+    return cuda_status(launch_decode_select(sh, scores, ids, st, true));
+}
+
+msa_status msa_sparse_attn_paged(const void *q, const void *k_pages, const void *v_pages,
+                                 const int32_t *page_table, int page_stride, int num_pages,
+                                 const int32_t *ids, float *out, float *lse, int Bt, int T,
+                                 int Hq, int Hkv, int d, int block, int K, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    if (!q || !k_pages || !v_pages || !page_table || !ids || !out || !lse)
+        return MSA_ERR_INVALID_ARG;
+    Shape sh;
+    msa_status s = validate(Bt, 1, T, Hq, Hkv, d, 64, block, K, false, true, &sh);
+    if (s != MSA_OK) return s;
+    if (page_stride < sh.N || num_pages < 1) return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) ||
+        (reinterpret_cast<uintptr_t>(page_table) & 3))
+        return MSA_ERR_INVALID_ARG;
+    const WsLayout L = layout_for(sh, true);
+    if ((s = check_ws(workspace, workspace_bytes, L)) != MSA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int *status = at<int>(workspace, L.status);
+    const int S = L.decode_splits;
+    float *po = at<float>(workspace, L.part_o);
+    float *pl = at<float>(workspace, L.part_lse);
+    const PageMap pm{page_table, page_stride, num_pages};
+    cudaError_t e = launch_decode_attn(sh, q, k_pages, v_pages, ids, po, pl, S, pm, status, st, true);
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    return cuda_status(launch_combine(sh, po, false, pl, ids, out, lse, S, st, true));
 }
 
 msa_status msa_device_status(void *workspace, void *stream) {

@@ -24,6 +24,16 @@ struct Shape {
     int G;  // Hq / Hkv
 };
 
+// Paged KV for decode: logical block j of sequence b is physical page
+// table[b * stride + j] of a store of `count` pages of `block` rows each
+// (k_idx pages [count][block][d_idx], K/V pages [count][block][Hkv][d]).
+// table == nullptr: contiguous [Bt][T] rows.
+struct PageMap {
+    const int32_t *table = nullptr;
+    int stride = 0;
+    int count = 0;
+};
+
 // One unit of work of the prefill attention kernel: the hit list of one
 // (sequence, block) pair, rows [start, start + count) of that list.
 struct AttnItem {

@@ -96,7 +96,8 @@ msa_status msa_sparse_attn_decode_noalloc(const void *q, const void *k, const vo
         dev_status = reinterpret_cast<int *>(b);
         if (cudaMemsetAsync(dev_status, 0, sizeof(int), st) != cudaSuccess) return MSA_ERR_CUDA;
     }
-    if (launch_decode_attn(sh, q, k, v, ids, part_o, part_lse, S, dev_status, st, false) != cudaSuccess)
+    if (launch_decode_attn(sh, q, k, v, ids, part_o, part_lse, S, PageMap{}, dev_status, st, false) !=
+        cudaSuccess)
         return MSA_ERR_CUDA;
     if (launch_combine(sh, part_o, false, part_lse, ids, out, lse, S, st, true) != cudaSuccess)
         return MSA_ERR_CUDA;

@@ -26,7 +26,8 @@ STATUS = {
 
 EXPORTED = ("msa_workspace_size", "msa_index_topk", "msa_select_invert", "msa_sparse_attn",
             "msa_index_topk_ev", "msa_sparse_attn_ev", "msa_device_status", "msa_status_string",
-            "msa_selftest_umma", "msa_sparse_attn_decode_noalloc")
+            "msa_selftest_umma", "msa_sparse_attn_decode_noalloc", "msa_index_topk_paged",
+            "msa_sparse_attn_paged")
 
 MAX_STAGES = 4
 
@@ -91,6 +92,10 @@ def load_library(path: str = LIB_PATH):
     lib.msa_sparse_attn_ev.restype = I
     lib.msa_sparse_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
     lib.msa_sparse_attn_decode_noalloc.restype = I
+    lib.msa_index_topk_paged.argtypes = [P, P, P, I, I, P, I, I, I, I, I, P, Z, P]
+    lib.msa_index_topk_paged.restype = I
+    lib.msa_sparse_attn_paged.argtypes = [P, P, P, P, I, I, P, P, P, I, I, I, I, I, I, I, P, Z, P]
+    lib.msa_sparse_attn_paged.restype = I
     lib.msa_selftest_umma.argtypes = [P, P, P, I, I, I, P, P]
     lib.msa_selftest_umma.restype = I
     _lib = lib
@@ -207,6 +212,59 @@ def sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ids: torch.Te
                                                      lse.data_ptr(), Bt, n_q, T, Hq, Hkv, d,
                                                      block, K, ws.ptr, ws.nbytes,
                                                      _stream(stream), _stage_events(events)))
+    return out, lse
+
+
+def index_topk_paged(q_idx: torch.Tensor, k_idx_pages: torch.Tensor, page_table: torch.Tensor,
+                     T: int, K: int, ws: Workspace, ids: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Decode index branch over paged index keys (msa_index_topk_paged):
+    q_idx [Bt, 1, d_idx], k_idx_pages [num_pages, block, d_idx] bf16,
+    page_table [Bt, page_stride] int32 -> ids [Bt, 1, K] int32."""
+    _dev(q_idx, torch.bfloat16, "q_idx")
+    _dev(k_idx_pages, torch.bfloat16, "k_idx_pages")
+    _dev(page_table, torch.int32, "page_table")
+    Bt, n_q, d_idx = q_idx.shape
+    num_pages, block, d2 = k_idx_pages.shape
+    if n_q != 1 or d2 != d_idx or page_table.dim() != 2 or page_table.shape[0] != Bt:
+        raise ValueError("paged index: q_idx [Bt, 1, d_idx], k_idx_pages [pages, block, d_idx], "
+                         "page_table [Bt, stride]")
+    if ids is None:
+        ids = torch.empty((Bt, 1, K), dtype=torch.int32, device=q_idx.device)
+    _dev(ids, torch.int32, "ids")
+    _check("msa_index_topk_paged", load_library().msa_index_topk_paged(
+        q_idx.data_ptr(), k_idx_pages.data_ptr(), page_table.data_ptr(), page_table.shape[1],
+        num_pages, ids.data_ptr(), Bt, T, d_idx, block, K, ws.ptr, ws.nbytes, _stream(stream)))
+    return ids
+
+
+def sparse_attn_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                      page_table: torch.Tensor, T: int, ids: torch.Tensor, ws: Workspace,
+                      out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                      stream=None):
+    """Decode sparse branch over paged K/V (msa_sparse_attn_paged): q [Bt, 1, Hq, d],
+    k_pages/v_pages [num_pages, block, Hkv, d] bf16, page_table [Bt, page_stride]
+    int32, ids [Bt, 1, K] -> (out [Bt, 1, Hq, d], lse [Bt, 1, Hq]) fp32."""
+    for t, name in ((q, "q"), (k_pages, "k_pages"), (v_pages, "v_pages")):
+        _dev(t, torch.bfloat16, name)
+    _dev(page_table, torch.int32, "page_table")
+    _dev(ids, torch.int32, "ids")
+    Bt, n_q, Hq, d = q.shape
+    num_pages, block, Hkv, d2 = k_pages.shape
+    K = ids.shape[-1]
+    if n_q != 1 or d2 != d or v_pages.shape != k_pages.shape or ids.shape != (Bt, 1, K) or \
+            page_table.dim() != 2 or page_table.shape[0] != Bt:
+        raise ValueError("paged attention: shapes do not match")
+    if out is None:
+        out = torch.empty((Bt, 1, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((Bt, 1, Hq), dtype=torch.float32, device=q.device)
+    _dev(out, torch.float32, "out")
+    _dev(lse, torch.float32, "lse")
+    _check("msa_sparse_attn_paged", load_library().msa_sparse_attn_paged(
+        q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), page_table.data_ptr(),
+        page_table.shape[1], num_pages, ids.data_ptr(), out.data_ptr(), lse.data_ptr(), Bt, T, Hq,
+        Hkv, d, block, K, ws.ptr, ws.nbytes, _stream(stream)))
     return out, lse
 
 

@@ -131,6 +131,35 @@ MSA_API msa_status msa_sparse_attn(const void *q, const void *k, const void *v,
                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Paged KV for decode [P4 section 3.2, "MSA 如何降低显存压力": page-managed
+ * KV cache; its 4-bit quantisation is not followed, KV stays raw bf16].
+ * Same computation as msa_index_topk / msa_sparse_attn for a decode step
+ * (n_q = 1, the query at t = T-1), with k_idx, K and V held in pages of
+ * `block` rows instead of contiguous [Bt][T] rows:
+ *   page_table  [Bt][page_stride] int32 (device): logical block j of
+ *               sequence b is physical page page_table[b*page_stride + j],
+ *               for j < N = ceil(T / block); page_stride >= N.
+ *   k_idx_pages [num_pages][block][d_idx] bf16;
+ *   k_pages, v_pages [num_pages][block][Hkv][d] bf16 (16-byte aligned).
+ * Rows past T in the last logical block are never read.  The caller owns
+ * all buffers; the workspace is msa_workspace_size(Bt, 1, T, ...).  A page id
+ * outside [0, num_pages) is skipped and reported as MSA_ERR_BAD_IDS through
+ * the status word (msa_device_status).  Host-detected errors as above.
+ */
+MSA_API msa_status msa_index_topk_paged(const void *q_idx, const void *k_idx_pages,
+                                        const int32_t *page_table, int page_stride,
+                                        int num_pages, int32_t *ids, int Bt, int T, int d_idx,
+                                        int block, int K, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
+MSA_API msa_status msa_sparse_attn_paged(const void *q, const void *k_pages, const void *v_pages,
+                                         const int32_t *page_table, int page_stride,
+                                         int num_pages, const int32_t *ids, float *out,
+                                         float *lse, int Bt, int T, int Hq, int Hkv, int d,
+                                         int block, int K, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+
+/*
  * Instrumented variants (profiling): the same work as msa_index_topk and
  * msa_sparse_attn, with optional CUDA events recorded on `stream`
  * immediately before (start[i]) and after (stop[i]) the kernels of stage i.

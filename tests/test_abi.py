@@ -89,6 +89,26 @@ def test_sparse_attn_host_validation(lib):
     assert call(*ok, 1, 1 << 20, 1 << 20, 128, 1, 128, 128, 4, FAKE, 1 << 50, None) == 2
 
 
+def test_paged_decode_host_validation(lib):
+    idx = lib.msa_index_topk_paged
+    # q_idx, k_idx_pages, page_table, stride, pages, ids, Bt, T, d_idx, block, K, ws, bytes, stream
+    assert idx(None, FAKE, FAKE, 8, 16, FAKE, 1, 512, 64, 64, 4, FAKE, 1 << 20, None) == 1
+    assert idx(FAKE, FAKE, FAKE, 7, 16, FAKE, 1, 512, 64, 64, 4, FAKE, 1 << 20, None) == 1  # stride < N
+    assert idx(FAKE, FAKE, FAKE, 8, 0, FAKE, 1, 512, 64, 64, 4, FAKE, 1 << 20, None) == 1   # no pages
+    assert idx(FAKE, FAKE, FAKE, 8, 16, FAKE, 1, 512, 96, 64, 4, FAKE, 1 << 20, None) == 2  # d_idx
+    assert idx(FAKE, FAKE, FAKE, 8, 16, FAKE, 1, 512, 64, 64, 4, FAKE, 16, None) == 3       # ws
+    att = lib.msa_sparse_attn_paged
+    ok = (FAKE,) * 4
+    # q, k_pages, v_pages, table, stride, pages, ids, out, lse, Bt, T, Hq, Hkv, d, block, K, ws...
+    assert att(*ok, 8, 16, FAKE, FAKE, None, 1, 512, 8, 2, 64, 64, 4, FAKE, 1 << 20, None) == 1
+    assert att(*ok, 7, 16, FAKE, FAKE, FAKE, 1, 512, 8, 2, 64, 64, 4, FAKE, 1 << 20, None) == 1
+    assert att(*ok, 8, 16, FAKE, FAKE, FAKE, 1, 512, 8, 3, 64, 64, 4, FAKE, 1 << 20, None) == 1
+    assert att(*ok, 8, 16, FAKE, FAKE, FAKE, 1, 512, 8, 2, 80, 64, 4, FAKE, 1 << 20, None) == 2
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    assert att(FAKE, FAKE, FAKE, odd, 8, 16, FAKE, FAKE, FAKE, 1, 512, 8, 2, 64, 64, 4, FAKE,
+               1 << 20, None) == 1  # page table not 4-byte aligned
+
+
 def test_select_invert_host_validation(lib):
     call = lib.msa_select_invert
     assert call(None, FAKE, FAKE, 1, 8, 8, 64, 4, FAKE, 1 << 20, None) == 1
