@@ -457,14 +457,15 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
 // out = sum_p exp(lse_p - LSE) o_p.  Weights are computed once into shared
 // memory; the partial rows are then streamed with 16-byte loads (several in
 // flight per thread).  Partial p = (slot s, split sp) is valid when
-// ids[row][s] >= 0 and its lse is finite; invalid partials are never used
-// (their memory may hold a previous call's data).
+// 0 <= ids[row][s] < N and its lse is finite; invalid partials are never used
+// (their memory may hold a previous call's data: the attention kernels write
+// no partial for an id outside [0, N)).
 // ------------------------------------------------------------------------
 template <typename PT, int D>
 __global__ void __launch_bounds__(256) lse_combine_kernel(
     const PT *__restrict__ part_o, const float *__restrict__ part_lse,
     const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
-    int K, int S, int HG, int G) {
+    int K, int S, int HG, int G, int N) {
     grid_dep_wait();  // inputs come from the previous kernel in the stream
     constexpr int VEC = 16 / sizeof(PT);  // elements per 16-byte load
     constexpr int NV = D / VEC;           // 16-byte loads per head row
@@ -478,7 +479,8 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
         const int pp = e / HG, hh = e % HG;
         const int s = pp / S;
         float l = -INFINITY;
-        if (ids[row * K + s] >= 0) l = part_lse[((row * K + s) * S + pp % S) * Hq + h0 + hh];
+        const int j = ids[row * K + s];
+        if (j >= 0 && j < N) l = part_lse[((row * K + s) * S + pp % S) * Hq + h0 + hh];
         wsm[e] = l;
     }
     __syncthreads();
@@ -546,7 +548,7 @@ template <typename PT, int D, int NW>
 __global__ void __launch_bounds__(32 * NW) lse_combine_split_kernel(
     const PT *__restrict__ part_o, const float *__restrict__ part_lse,
     const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
-    int K, int S) {
+    int K, int S, int N) {
     grid_dep_wait();  // inputs come from the previous kernel in the stream
     constexpr int PER = D / 32;  // elements per lane
     extern __shared__ float wsm[];                // [P] weights, then [NW][D] sums
@@ -559,7 +561,8 @@ __global__ void __launch_bounds__(32 * NW) lse_combine_split_kernel(
     for (int pp = tid; pp < P; pp += blockDim.x) {
         const int si = pp / S;
         float l = -INFINITY;
-        if (ids[row * K + si] >= 0) l = part_lse[((row * K + si) * S + pp % S) * Hq + h];
+        const int j = ids[row * K + si];
+        if (j >= 0 && j < N) l = part_lse[((row * K + si) * S + pp % S) * Hq + h];
         wsm[pp] = l;
     }
     __syncthreads();
@@ -923,7 +926,7 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
         cudaFuncSetAttribute(lse_combine_split_kernel<float, DD, NWW>,                            \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
         return launch_ex(lse_combine_split_kernel<float, DD, NWW>, grid, dim3(32 * NWW), smem, st, \
-                         pdl, po, part_lse, ids, out, lse, sh.Hq, sh.K, S);                        \
+                         pdl, po, part_lse, ids, out, lse, sh.Hq, sh.K, S, sh.N);                  \
     } while (0)
         if (sh.d == 128) {
             if (wide) MSA_COMBINE_SPLIT(128, 8);
@@ -949,7 +952,7 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
         e = launch_ex(lse_combine_kernel<PT, DD>, grid, dim3(threads), smem, st, pdl,             \
                       static_cast<const PT *>(part_o), part_lse, ids, out, lse, sh.Hq, sh.K, S,   \
-                      HG, part_bf16 ? sh.G : 0);                                                  \
+                      HG, part_bf16 ? sh.G : 0, sh.N);                                            \
     } while (0)
     cudaError_t e = cudaSuccess;
     if (part_bf16) {

@@ -143,6 +143,7 @@ bool make_tmap(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dim
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
 
 // Record the start/stop event of stage i (if the caller supplied one).
 void mark(const msa_stage_events *ev, int i, bool start, cudaStream_t st) {
@@ -176,7 +177,7 @@ msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids,
     Shape sh;
     msa_status s = validate(Bt, n_q, T, 1, 1, 64, d_idx, block, K, true, false, &sh);
     if (s != MSA_OK) return s;
-    if (!aligned16(q_idx) || !aligned16(k_idx)) return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned4(ids)) return MSA_ERR_INVALID_ARG;
     const WsLayout L = layout_for(sh, false);
     if ((s = check_ws(workspace, workspace_bytes, L)) != MSA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -216,6 +217,7 @@ msa_status msa_select_invert(const int32_t *ids, int32_t *row_ptr, int32_t *entr
     msa_status s = validate(Bt, n_q, T, 1, 1, 64, 64, block, K, false, false, &sh);
     if (s != MSA_OK) return s;
     if (sh.N > kMaxBlocksPrefill) return MSA_ERR_UNSUPPORTED;
+    if (!aligned4(ids) || !aligned4(row_ptr) || !aligned4(entries)) return MSA_ERR_INVALID_ARG;
     const WsLayout L = layout_for(sh, false);
     if ((s = check_ws(workspace, workspace_bytes, L)) != MSA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -241,7 +243,11 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     Shape sh;
     msa_status s = validate(Bt, n_q, T, Hq, Hkv, d, 64, block, K, false, true, &sh);
     if (s != MSA_OK) return s;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return MSA_ERR_INVALID_ARG;
+    // the combine writes out with 16-byte stores; ids and lse are read and
+    // written as 4-byte words
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(ids) ||
+        !aligned4(lse))
+        return MSA_ERR_INVALID_ARG;
     const WsLayout L = layout_for(sh, true);
     if ((s = check_ws(workspace, workspace_bytes, L)) != MSA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -301,7 +307,7 @@ msa_status msa_index_topk_paged(const void *q_idx, const void *k_idx_pages,
     msa_status s = validate(Bt, 1, T, 1, 1, 64, d_idx, block, K, true, false, &sh);
     if (s != MSA_OK) return s;
     if (page_stride < sh.N || num_pages < 1) return MSA_ERR_INVALID_ARG;
-    if (!aligned16(q_idx) || !aligned16(k_idx_pages) || (reinterpret_cast<uintptr_t>(page_table) & 3))
+    if (!aligned16(q_idx) || !aligned16(k_idx_pages) || !aligned4(page_table) || !aligned4(ids))
         return MSA_ERR_INVALID_ARG;
     const WsLayout L = layout_for(sh, false);
     if ((s = check_ws(workspace, workspace_bytes, L)) != MSA_OK) return s;
@@ -327,8 +333,8 @@ msa_status msa_sparse_attn_paged(const void *q, const void *k_pages, const void 
     msa_status s = validate(Bt, 1, T, Hq, Hkv, d, 64, block, K, false, true, &sh);
     if (s != MSA_OK) return s;
     if (page_stride < sh.N || num_pages < 1) return MSA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) ||
-        (reinterpret_cast<uintptr_t>(page_table) & 3))
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out) ||
+        !aligned4(page_table) || !aligned4(ids) || !aligned4(lse))
         return MSA_ERR_INVALID_ARG;
     const WsLayout L = layout_for(sh, true);
     if ((s = check_ws(workspace, workspace_bytes, L)) != MSA_OK) return s;

@@ -58,9 +58,12 @@ msa_status msa_sparse_attn_decode_noalloc(const void *q, const void *k, const vo
     if (K > kMaxK || !(d == 64 || d == 128) || !(block == 32 || block == 64 || block % 128 == 0) ||
         128 % (Hq / Hkv) != 0 || static_cast<long long>(Bt) * T >= (1ll << 31))
         return MSA_ERR_UNSUPPORTED;
+    // q, k, v are read and out is written with 16-byte accesses; ids and lse
+    // as 4-byte words
     const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                          reinterpret_cast<uintptr_t>(v);
-    if (mis & 15) return MSA_ERR_INVALID_ARG;
+                          reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
+    if ((mis & 15) || ((reinterpret_cast<uintptr_t>(ids) | reinterpret_cast<uintptr_t>(lse)) & 3))
+        return MSA_ERR_INVALID_ARG;
 
     Shape sh;
     sh.Bt = Bt;

@@ -43,8 +43,11 @@
  *    multiple of 128; 1 <= K <= 32; 128 % (Hq/Hkv) == 0; N <= 8192;
  *    Bt*T < 2^31, Bt*n_q*K < 2^31 and Bt*n_q*Hq*d < 2^34 (the attention
  *    calls address q in 16-byte units with 32-bit offsets).  Anything else
- *    returns MSA_ERR_UNSUPPORTED before any work is enqueued.  Tensor base
- *    pointers must be 16-byte aligned (MSA_ERR_INVALID_ARG otherwise).
+ *    returns MSA_ERR_UNSUPPORTED before any work is enqueued.
+ *  - Alignment (MSA_ERR_INVALID_ARG otherwise, nothing enqueued): q_idx,
+ *    k_idx, q, k, v (and their paged stores) and out must be 16-byte aligned
+ *    (they are read or written in 16-byte pieces); ids, lse, row_ptr,
+ *    entries and page tables 4-byte aligned.
  *  - Errors found on the host return immediately (nothing enqueued).  Errors a
  *    kernel finds (an id outside [-1, N), a bounded wait that expired) are
  *    OR-ed into a sticky status word at the start of the workspace; kernels
@@ -119,7 +122,8 @@ MSA_API msa_status msa_select_invert(const int32_t *ids, int32_t *row_ptr, int32
  * attention over the keys of the selected blocks (causal inside the own block),
  * scale 1/sqrt(d), raw bf16 KV.  Writes out and lse (layouts above).
  * ids must hold, per row, distinct block ids in [0, N) or -1; an id greater
- * than own(t) contributes no key.  Prefill (n_q > 1): inversion, a
+ * than own(t) contributes no key; an id outside [-1, N) is skipped (it
+ * contributes no key either) and reported as MSA_ERR_BAD_IDS.  Prefill (n_q > 1): inversion, a
  * KV-block-outer tcgen05 kernel that loads each selected KV block into shared
  * memory and gathers its hit queries, then a log-sum-exp combine of the per
  * slot partials.  Decode (n_q == 1): a split-K kernel over the selected blocks,
@@ -208,7 +212,9 @@ MSA_API msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *
  *     1M-context decode, Bt 4, K 8, block 512, Hq 64, d 128, needs 8.5 MB.)
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture begins.
+ *     stream capture begins.  The cached address belongs to the device's
+ *     primary context: after cudaDeviceReset, or when calling from another
+ *     driver context on the same device, it is stale and must not be used.
  *   - Every call uses the same array, which keeps the contents of the last
  *     call.  Calls whose kernels overlap on the GPU (two streams, or two host
  *     threads) race on it and must be serialised by the caller.

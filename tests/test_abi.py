@@ -89,6 +89,34 @@ def test_sparse_attn_host_validation(lib):
     assert call(*ok, 1, 1 << 20, 1 << 20, 128, 1, 128, 128, 4, FAKE, 1 << 50, None) == 2
 
 
+def test_misaligned_outputs_rejected_on_host(lib):
+    # out is written with 16-byte stores, ids and lse as 4-byte words: a
+    # misaligned pointer is rejected before anything is enqueued
+    att = lib.msa_sparse_attn
+    odd4 = ctypes.c_void_p((1 << 20) + 4)   # 4-byte but not 16-byte aligned
+    odd2 = ctypes.c_void_p((1 << 20) + 2)   # not 4-byte aligned
+    # q, k, v, ids, out, lse, Bt, n_q, T, Hq, Hkv, d, block, K, ws, bytes, stream
+    args = (1, 8, 8, 8, 2, 64, 64, 4, FAKE, 1 << 30, None)
+    assert att(FAKE, FAKE, FAKE, FAKE, odd4, FAKE, *args) == 1      # out
+    assert att(FAKE, FAKE, FAKE, FAKE, FAKE, odd2, *args) == 1      # lse
+    assert att(FAKE, FAKE, FAKE, odd2, FAKE, FAKE, *args) == 1      # ids
+    dec = (1, 1, 8, 8, 2, 64, 64, 4, FAKE, 1 << 30, None)           # decode shape
+    assert att(FAKE, FAKE, FAKE, FAKE, odd4, FAKE, *dec) == 1
+    idx = lib.msa_index_topk
+    assert idx(FAKE, FAKE, odd2, 1, 8, 8, 64, 64, 4, FAKE, 1 << 20, None) == 1  # ids
+    inv = lib.msa_select_invert
+    assert inv(FAKE, odd2, FAKE, 1, 8, 8, 64, 4, FAKE, 1 << 20, None) == 1      # row_ptr
+    na = lib.msa_sparse_attn_decode_noalloc
+    # q, k, v, ids, out, lse, Bt, T, Hq, Hkv, d, block, K, status, stream
+    assert na(FAKE, FAKE, FAKE, FAKE, odd4, FAKE, 1, 1000, 8, 2, 64, 64, 4, None, None) == 1
+    assert na(FAKE, FAKE, FAKE, FAKE, FAKE, odd2, 1, 1000, 8, 2, 64, 64, 4, None, None) == 1
+    assert na(FAKE, FAKE, FAKE, odd2, FAKE, FAKE, 1, 1000, 8, 2, 64, 64, 4, None, None) == 1
+    pa = lib.msa_sparse_attn_paged
+    # q, k_pages, v_pages, table, stride, pages, ids, out, lse, Bt, T, Hq, Hkv, d, block, K, ...
+    assert pa(FAKE, FAKE, FAKE, FAKE, 8, 16, FAKE, odd4, FAKE, 1, 512, 8, 2, 64, 64, 4, FAKE,
+              1 << 20, None) == 1
+
+
 def test_paged_decode_host_validation(lib):
     idx = lib.msa_index_topk_paged
     # q_idx, k_idx_pages, page_table, stride, pages, ids, Bt, T, d_idx, block, K, ws, bytes, stream

@@ -79,6 +79,19 @@ def test_decode_bad_ids_reported():
     x = make_inputs(w, device="cuda")
     ids = torch.tensor([[[0, 3, 15, 99]], [[-7, 1, 2, 15]]], dtype=torch.int32, device="cuda")
     ws = msa.Workspace.for_shape(w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K)
-    msa.sparse_attn(x["q"], x["k"], x["v"], ids, w.block, ws)
+    out, lse = msa.sparse_attn(x["q"], x["k"], x["v"], ids, w.block, ws)
     assert msa.device_status(ws) == 6  # MSA_ERR_BAD_IDS
     assert msa.device_status(ws) == 0  # read-and-clear
+    # the skipped ids contribute no key: each row equals the oracle over the rest
+    from oracle import oracle
+    hx = {k: host(v) for k, v in x.items()}
+    o_ref, l_ref = oracle.sparse_attn(hx["q"], hx["k"], hx["v"], host(ids).reshape(-1, w.K), w.Bt,
+                                      1, w.T, w.Hq, w.Hkv, w.d, w.block, w.K)
+    assert_close(host(out).numpy().reshape(o_ref.shape), o_ref, "out")
+    assert_close(host(lse).numpy().reshape(l_ref.shape), l_ref, "lse")
+
+
+def test_decode_many_rows_and_heads():
+    # Bt * Hq >= 4096: the combine takes the row-parallel kernel (fp32
+    # partials, two splits per 128-key block) instead of the split combine
+    _decode_case(Workload("dec_wide", 64, 1, 2048, 64, 8, 128, 128, 4, 64))

@@ -168,3 +168,43 @@ def test_prefill_bad_ids_reported():
     out, lse = msa.sparse_attn(x["q"], x["k"], x["v"], ids, w.block, ws)
     assert msa.device_status(ws) == 6  # MSA_ERR_BAD_IDS
     assert torch.isfinite(out[0, 100]).all()
+
+
+def _with_odd_ids(w, ids, beyond_own=True, out_of_range=True):
+    """A copy of a selection with, in some rows, one slot replaced by a block
+    after the row's own block (such a block holds no key at or before t) and,
+    in other rows, one slot replaced by an id >= N (skipped and reported)."""
+    h = ids.cpu().clone().view(-1, w.K)
+    N = w.n_blocks
+    for r in range(h.shape[0]):
+        t = w.T - w.n_q + r % w.n_q
+        own = t // w.block
+        row = h[r].tolist()
+        # the slot to replace: a -1 pad if there is one, else a non-own block
+        cand = [s for s in range(w.K) if row[s] == -1] or [s for s in range(w.K) if row[s] != own]
+        if not cand:
+            continue
+        s = cand[r % len(cand)]
+        if beyond_own and r % 3 == 0 and own + 1 < N:
+            later = [j for j in range(own + 1, N) if j not in row]
+            h[r, s] = later[r % len(later)]
+        elif out_of_range and r % 3 == 1:
+            h[r, s] = N + r % 5
+    return h.view_as(ids).to(ids.device)
+
+
+@pytest.mark.parametrize("out_of_range", [False, True], ids=["beyond_own", "beyond_own_and_N"])
+def test_prefill_ids_beyond_own_and_out_of_range(out_of_range):
+    # a block after own(t) contributes no key; an id >= N is skipped (and
+    # reported): either way the row equals the attention over its other ids
+    from block_sparse_long_05_b200 import msa
+    lib_ready()
+    for w in (Workload("pf_odd_ids", 1, 1024, 1024, 8, 2, 64, 64, 4, 64),
+              Workload("pf_odd_ids_b512", 1, 3000, 3000, 8, 4, 128, 512, 3, 64)):
+        x = make_inputs(w, device="cuda")
+        ids = _with_odd_ids(w, random_selection(w, device="cuda"), out_of_range=out_of_range)
+        ws = _ws(w)
+        out, lse = msa.sparse_attn(x["q"], x["k"], x["v"], ids, w.block, ws)
+        assert msa.device_status(ws) == (6 if out_of_range else 0)
+        rows = torch.arange(w.Bt * w.n_q, dtype=torch.int64)
+        _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)

@@ -55,3 +55,27 @@ def test_noalloc_rejects_oversized_shape():
     rc = lib.msa_sparse_attn_decode_noalloc(fake, fake, fake, fake, fake, fake, w.Bt, w.T, w.Hq,
                                             w.Hkv, w.d, w.block, w.K, None, None)
     assert rc == 3  # MSA_ERR_WORKSPACE, nothing enqueued
+
+
+def test_noalloc_without_status_and_with_many_rows():
+    # status = NULL (the library clears and uses a word of its own scratch),
+    # and a shape with Bt * Hq >= 4096, where the combine takes its
+    # row-parallel kernel; two calls in a row, against the workspace path
+    from block_sparse_long_05_b200 import msa
+    from block_sparse_long_05_b200.inputs import Workload, make_inputs
+    lib_ready()
+    for w in (Workload("noalloc_nostatus", 3, 1, 5000, 16, 2, 128, 128, 8, 64),
+              Workload("noalloc_wide", 64, 1, 2048, 64, 8, 128, 128, 3, 64)):
+        x = make_inputs(w, device="cuda")
+        ws = msa.Workspace.for_shape(w.Bt, 1, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K)
+        ids = msa.index_topk(x["q_idx"], x["k_idx"], w.block, w.K, ws)
+        ref_out, ref_lse = msa.sparse_attn(x["q"], x["k"], x["v"], ids, w.block, ws)
+        assert msa.device_status(ws) == 0
+        for call in range(2):
+            out = torch.full_like(ref_out, float("nan"))
+            lse = torch.full_like(ref_lse, float("nan"))
+            msa.sparse_attn_decode_noalloc(x["q"], x["k"], x["v"], ids, w.block, out=out,
+                                           lse=lse, status=None)
+            torch.cuda.synchronize()
+            _compare(out, ref_out, f"{w.name} out, call {call}")
+            _compare(lse, ref_lse, f"{w.name} lse, call {call}")
