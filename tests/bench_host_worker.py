@@ -3,8 +3,10 @@ events and the clock sampler replaced by fakes, on small stand-ins for the
 default prefill and decode workloads; prints the JSON line.  Launched in its
 own process by tests/test_bench_model.py (it patches torch for that process).
 
-argv[1]: "flush" (small steps: L2 flushed between timed steps) or "noflush"
-(the L2 threshold set to one byte: back-to-back timing)."""
+argv[1]: "flush" (small steps: L2 flushed between timed steps), "noflush"
+(the L2 threshold set to one byte: back-to-back timing) or "heads" (run
+under torch.distributed.run with gloo ranks: the kv-head-sharded long
+prefill, its ids all-gathered between the ranks)."""
 import json
 import os
 import sys
@@ -87,12 +89,48 @@ def main():
     msa.sparse_attn = fake_sparse_attn
     msa.device_status = lambda ws, stream=None: 0
     W = inputs.Workload
-    inputs.WORKLOADS[bench.DEFAULT_WORKLOAD] = W(bench.DEFAULT_WORKLOAD, 1, 256, 256, 8, 2, 64, 32, 4, 64)
-    inputs.WORKLOADS[bench.SECONDARY_DECODE] = W(bench.SECONDARY_DECODE, 4, 1, 4096, 8, 2, 64, 128, 4, 64)
+    # small stand-ins with each workload's kind (prefill / decode)
+    small = {"tiny_prefill_T4096": W("tiny_prefill_T4096", 1, 128, 128, 8, 2, 64, 32, 4, 64),
+             "prefill_T65536": W("prefill_T65536", 1, 256, 256, 8, 2, 64, 32, 4, 64),
+             "decode_32x131072": W("decode_32x131072", 3, 1, 2048, 8, 2, 64, 128, 4, 64),
+             "long_prefill_T262144": W("long_prefill_T262144", 1, 256, 256, 8, 2, 64, 64, 4, 64),
+             "decode_4x1048576": W("decode_4x1048576", 4, 1, 4096, 8, 2, 64, 128, 4, 64)}
+    inputs.WORKLOADS.update(small)
     if sys.argv[1] == "noflush":
         bench.L2_BYTES = 1
     args = types.SimpleNamespace(workload=bench.DEFAULT_WORKLOAD, steps=3, warmup=1, no_e2e=True,
-                                 no_cpu_baseline=True, no_decode=False, cpu_seconds=1.0)
+                                 no_cpu_baseline=True, no_decode=False, cpu_seconds=1.0,
+                                 only=False)
+    if sys.argv[1] == "heads":
+        import datetime
+        import torch.distributed as dist
+        rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        seen = []
+        real_attn = msa.sparse_attn
+
+        def recording_attn(q, k, v, ids, block, ws, **kw):
+            seen.append((tuple(q.shape), tuple(k.shape), ids.clone()))
+            return real_attn(q, k, v, ids, block, ws, **kw)
+        msa.sparse_attn = recording_attn
+        try:
+            line = bench.run_msa(args, rank, world, rank)
+            q_shape, k_shape, ids = seen[-1]
+            mine = torch.tensor([float(ids.long().sum()), float(q_shape[2]), float(k_shape[2])],
+                                dtype=torch.float64)
+            parts = [torch.zeros_like(mine) for _ in range(world)]
+            dist.all_gather(parts, mine)
+            w = inputs.WORKLOADS[bench.DEFAULT_WORKLOAD]
+            ref = torch.empty((1, w.n_q, w.K), dtype=torch.int32)
+            fake_index_topk(torch.empty((1, w.n_q, w.d_idx)), torch.empty((1, w.T, w.d_idx)),
+                            w.block, w.K, None, ids=ref)
+            if rank == 0:
+                line["_ranks"] = [p.tolist() for p in parts]
+                line["_ids_sum"] = float(ref.long().sum())
+                print(json.dumps(line))
+        finally:
+            dist.destroy_process_group()
+        return
     print(json.dumps(bench.run_msa(args, 0, 1, 0)))
 
 

@@ -71,18 +71,62 @@ def _host_run(mode):
 def test_bench_line_structure_with_and_without_l2_flush():
     """bench.py's measurement logic end to end on the CPU (library, events and
     clocks faked): the JSON line carries every key the benchmark contract
-    names, for both timing paths, with both decode secondaries."""
+    names, for both timing paths, with every workload under "configs"."""
     for mode, l2_word in (("flush", "flushed"), ("noflush", "no flush")):
         line = _host_run(mode)
         for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
                     "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
-                    "gpu_launches", "roofline", "clocks", "decode", "decode_at_T"):
+                    "gpu_launches", "roofline", "clocks", "decode_at_T", "configs", "kernels"):
             assert key in line, (mode, key)
+        assert line["config"]["workload"] == bench.DEFAULT_WORKLOAD
         assert l2_word in line["config"]["l2"], (mode, line["config"]["l2"])
         assert line["gpu_launches"] == 8 * line["steps"]
-        for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        for key in ("bound", "achieved", "peak", "unit", "frac", "traffic", "frac_sustained"):
             assert key in line["roofline"], key
+        # the tensor-core fraction is taken against the burst peak
+        assert abs(line["roofline"]["frac"] * line["roofline"]["peak"] -
+                   line["roofline"]["achieved"]) < 1e-6 * line["roofline"]["achieved"]
         assert "error" not in line["decode_at_T"], line["decode_at_T"]
         assert line["decode_at_T"]["workload"] == f"decode_1x{line['config']['T']}"
+        # every workload of the hot path, each with its own numbers
+        assert sorted(line["configs"]) == sorted(bench.CONFIGS)
+        for name, c in line["configs"].items():
+            assert "error" not in c, (name, c)
+            for key in ("value", "ms_per_step", "stage_ms", "roofline"):
+                assert key in c, (name, key)
+            exp_bound = "hbm" if name.startswith("decode") else "tensor"
+            assert c["roofline"]["bound"] == exp_bound, (name, c["roofline"])
         if mode == "flush":  # fake events tick 0.25 ms per record: one step = 0.25 ms
             assert abs(line["ms_per_step"] - 0.25) < 1e-9
+
+
+def test_bench_head_sharded_prefill_on_two_gloo_ranks():
+    """bench.py's kv-head-sharded long prefill on two gloo ranks (library
+    faked): each rank holds half of the heads, and the ids every rank's
+    sparse branch sees, all-gathered from the two row ranges, are the full
+    selection; the line reports strong scaling over 2 GPUs."""
+    import json
+    import os
+    import socket
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr=127.0.0.1", f"--master-port={port}",
+           os.path.join(root, "tests", "bench_host_worker.py"), "heads"]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=600,
+                       env=dict(os.environ, OMP_NUM_THREADS="1"))
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["scaling"] == "strong"
+    assert "kv-head" in line["config"]["parallelism"]
+    assert "gather" in line["stage_ms"]
+    assert "configs" not in line  # the other workloads are timed at one GPU only
+    for ids_sum, hq, hkv in line["_ranks"]:
+        assert ids_sum == line["_ids_sum"]       # the full selection on every rank
+        assert hq == line["config"]["Hq"] // 2 and hkv == line["config"]["Hkv"] // 2
