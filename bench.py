@@ -58,6 +58,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode step at each prefill workload's context")
+    ap.add_argument("--no-int8", action="store_true",
+                    help="skip the variant of each step with the int8 index path")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample (headline)")
     return ap.parse_args(argv)
@@ -241,6 +243,7 @@ class Problem:
         else:
             seed = rank_seed(w, rank) if mode == "seq" else w.seed
             self.x = make_inputs(w, device=dev, seed=seed)
+        self.int8_index = False  # index branch on int8 copies of the (integer) index keys
         self.Hq = (self.hk1 - self.hk0) * w.G
         self.Hkv = self.hk1 - self.hk0
         self.ws = msa.Workspace.for_shape(w.Bt, w.n_q, w.T, self.Hq, self.Hkv, w.d, w.d_idx,
@@ -273,10 +276,14 @@ class Problem:
         x = x or self.x
         y = y or self.y
         ev_idx, ev_attn, ev_gather = ev if ev else (None, None, None)
+        index = msa.index_topk
+        qi, ki = x["q_idx"], x["k_idx"]
+        if self.int8_index:
+            index, qi, ki = msa.index_topk_i8, x["q_idx8"], x["k_idx8"]
         if self.mode == "heads":
             if self.r1 > self.r0:
-                msa.index_topk(x["q_idx"], x["k_idx"], w.block, w.K, self.ws, ids=self.ids_local,
-                               stream=stream, events=ev_idx)
+                index(qi, ki, w.block, w.K, self.ws, ids=self.ids_local, stream=stream,
+                      events=ev_idx)
             ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
             with ctx:
                 if ev_gather:
@@ -286,10 +293,17 @@ class Problem:
                 if ev_gather:
                     ev_gather[1].record()
         else:
-            msa.index_topk(x["q_idx"], x["k_idx"], w.block, w.K, self.ws, ids=self.ids,
-                           stream=stream, events=ev_idx)
+            index(qi, ki, w.block, w.K, self.ws, ids=self.ids, stream=stream, events=ev_idx)
         msa.sparse_attn(x["q"], x["k"], x["v"], self.ids, w.block, self.ws, out=y["out"],
                         lse=y["lse"], stream=stream, events=ev_attn)
+
+    def use_int8_index(self):
+        """Switch the step to the int8 index path (msa_index_topk_i8) on int8
+        copies of the index keys (exact: the keys are small integers)."""
+        import torch
+        self.x["q_idx8"] = self.x["q_idx"].to(torch.int8)
+        self.x["k_idx8"] = self.x["k_idx"].to(torch.int8)
+        self.int8_index = True
 
     def touched_bytes(self):
         """Bytes one step reads and writes (to decide whether L2 must be
@@ -297,7 +311,8 @@ class Problem:
         w = self.w
         if w.is_decode:
             return sum(decode_bytes(w, self.ids, self.Hq, self.Hkv))
-        inputs = sum(t.numel() * t.element_size() for t in self.x.values())
+        inputs = sum(t.numel() * t.element_size() for k, t in self.x.items()
+                     if k not in ("q_idx8", "k_idx8"))
         partials = w.Bt * w.n_q * w.K * self.Hq * (w.d * 2 + 4)
         return inputs + partials + self.y["out"].numel() * 4
 
@@ -565,6 +580,40 @@ def roofline(w, prob, r, peaks, peak_src, traffic):
     return roof, kernels
 
 
+def measure_int8_index(w, prob, r, steps, warmup, peaks, peak_src):
+    """The same step with the index branch on int8 index keys
+    (msa_index_topk_i8); its ids must equal the bf16 path's."""
+    import torch
+    ids_bf16 = prob.ids.clone()
+    prob.use_int8_index()
+    try:
+        ri = measure(prob, steps, warmup, False)
+    finally:
+        prob.int8_index = False
+    sm = ri["stage_ms"]
+    obj = {"ms_per_step": ri["ms"], "value": w.Bt * w.n_q / (ri["ms"] / 1e3), "unit": UNIT,
+           "stage_ms": {k: round(v, 4) for k, v in sm.items()},
+           "ids_equal_bf16_path": bool(torch.equal(prob.ids, ids_bf16))}
+    t = sm.get("index0", 0.0)
+    if t > 0:
+        if w.is_decode:
+            scan_b = decode_bytes(w, prob.ids)[0] // 2  # int8 keys: half the bytes
+            obj["index_kernel"] = {"kernel": "decode_index_scan_kernel (int8)", "ms": round(t, 4),
+                                   "bound": "hbm", "achieved": scan_b / (t / 1e3) / 1e9,
+                                   "unit": "GB/s",
+                                   "frac": scan_b / (t / 1e3) / 1e9 / float(peaks["hbm_gbs"])}
+        else:
+            peak8 = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+            ach = 2.0 * index_macs(w) / (t / 1e3) / 1e12
+            obj["index_kernel"] = {"kernel": "prefill_index_kernel (kind::i8)", "ms": round(t, 4),
+                                   "bound": "tensor", "achieved": ach, "unit": "TOP/s",
+                                   "peak": peak8, "frac": ach / peak8,
+                                   "peak_note": f"int8 dense = 2 x the bf16 burst of {peak_src} "
+                                                "(nominal 4.5 / 2.25 PFLOP/s ratio)"}
+    del prob.x["q_idx8"], prob.x["k_idx8"]
+    return obj
+
+
 def bench_workload(w, args, rank, world, dev, peaks, peak_src, traffic, mode, steps, warmup,
                    with_e2e, decode_at_T, cpu_seconds):
     """Measure one workload; returns its JSON object (the headline's fields
@@ -575,6 +624,9 @@ def bench_workload(w, args, rank, world, dev, peaks, peak_src, traffic, mode, st
     r["pairs"] = attended_pairs(prob.ids, w)
     roof, kernels = roofline(w, prob, r, peaks, peak_src, traffic)
     tokens = w.Bt * w.n_q * (world if mode == "seq" else 1)
+    with_i8 = mode == "whole" and not getattr(args, "no_int8", False)
+    if with_i8:
+        obj_i8 = measure_int8_index(w, prob, r, steps, warmup, peaks, peak_src)
     obj = {"workload": w.name, "value": tokens / (r["ms"] / 1e3), "unit": UNIT,
            "ms_per_step": r["ms"], "stage_ms": {k: round(v, 4) for k, v in r["stage_ms"].items()},
            "roofline": roof, "kernels": kernels, "gpu_launches": r["launches"],
@@ -586,6 +638,8 @@ def bench_workload(w, args, rank, world, dev, peaks, peak_src, traffic, mode, st
         obj["step_frac_of_8tbs_nominal"] = (scan_b + kv_b) / (r["ms"] / 1e3) / 1e9 / 8000.0
     else:
         obj["attended_pairs"] = r["pairs"]
+    if with_i8:
+        obj["int8_index"] = obj_i8
     if "e2e" in r:
         e = r["e2e"]
         obj["e2e"] = {"value": tokens / (e["ms"] / 1e3), "unit": UNIT, "ms_per_step": e["ms"],

@@ -16,7 +16,7 @@ namespace msa {
 // are skipped and reported in *status
 cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k_idx,
                                float *block_scores, const PageMap &pm, int *status, int num_sms,
-                               cudaStream_t st);
+                               cudaStream_t st, bool int8_keys = false);
 // pdl: allow programmatic dependent launch after the previous kernel in st
 // (the kernel waits for it before reading its results)
 cudaError_t launch_decode_select(const Shape &sh, const float *block_scores, int32_t *ids,
@@ -38,9 +38,12 @@ size_t selftest_smem_bytes(int N, int Kd);
 cudaError_t launch_selftest_umma(const CUtensorMap &tm_a, const CUtensorMap &tm_b, float *C,
                                  int N, int Kd, int b_mn_major, int a_tmem, int *status,
                                  cudaStream_t st);
-size_t prefill_index_smem_bytes(int d_idx);
+size_t prefill_index_smem_bytes(int d_idx, int elem_bytes);
+// int8_keys: q_idx / k_idx are signed 8-bit integers (tcgen05 kind::i8)
+// instead of bf16 (kind::f16)
 cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                                 int32_t *ids, int *status, int num_sms, cudaStream_t st);
+                                 int32_t *ids, int *status, int num_sms, cudaStream_t st,
+                                 bool int8_keys);
 size_t prefill_attn_smem_bytes(const Shape &sh);
 int prefill_attn_rows_per_item(int G);
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,

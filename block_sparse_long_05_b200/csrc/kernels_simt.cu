@@ -64,13 +64,43 @@ __device__ __forceinline__ uint4 ld_stream16(const uint4 *p) {
     return v;
 }
 
-template <int D_IDX>
+// Dot product of one 16-byte piece of a key row with this lane's piece of the
+// query: 8 bf16 products in fp32, or 16 signed 8-bit products in exact
+// integer arithmetic (dp4a).
+struct ScanBf16 {
+    static constexpr int EPL = 8;  // elements per 16-byte load
+    float q[8];
+    __device__ void load_q(const void *p) { bf16x8_to_f32(*reinterpret_cast<const uint4 *>(p), q); }
+    __device__ float dot(const uint4 &u) const {
+        float kf[8];
+        bf16x8_to_f32(u, kf);
+        float sc = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sc = fmaf(q[e], kf[e], sc);
+        return sc;
+    }
+};
+struct ScanS8 {
+    static constexpr int EPL = 16;
+    uint4 q;
+    __device__ void load_q(const void *p) { q = *reinterpret_cast<const uint4 *>(p); }
+    __device__ float dot(const uint4 &u) const {
+        int acc = __dp4a(static_cast<int>(u.x), static_cast<int>(q.x), 0);
+        acc = __dp4a(static_cast<int>(u.y), static_cast<int>(q.y), acc);
+        acc = __dp4a(static_cast<int>(u.z), static_cast<int>(q.z), acc);
+        acc = __dp4a(static_cast<int>(u.w), static_cast<int>(q.w), acc);
+        return static_cast<float>(acc);  // |partial| <= 16 * 2^14: exact
+    }
+};
+
+template <int D_IDX, typename SC>
 __global__ void __launch_bounds__(256) decode_index_scan_kernel(
-    const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16 *__restrict__ k_idx,
+    const void *__restrict__ q_idx_v, const void *__restrict__ k_idx_v,
     float *__restrict__ block_scores, int Bt, int T, int block, int own, int N, int rw, int bpc,
     PageMap pm, int *__restrict__ status) {
     // rw: rows per warp (a warp's rows lie in one block); bpc: blocks per CTA
-    constexpr int LPR = D_IDX / 8;  // lanes per key row
+    constexpr int EB = 16 / SC::EPL;  // bytes per element
+    constexpr int LPR = D_IDX / SC::EPL;  // lanes per key row
     constexpr int RPL = 32 / LPR;   // key rows per warp load
     constexpr int UNR = 16;         // loads in flight per warp
     __shared__ float wmax[8];
@@ -96,11 +126,13 @@ __global__ void __launch_bounds__(256) decode_index_scan_kernel(
     }
     if (active) {
         const int b = static_cast<int>(item / own);
-        float qv[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(q_idx + static_cast<long long>(b) * D_IDX + part * 8), qv);
+        const unsigned char *q_idx = static_cast<const unsigned char *>(q_idx_v);
+        const unsigned char *k_idx = static_cast<const unsigned char *>(k_idx_v);
+        SC qv;
+        qv.load_q(q_idx + (static_cast<long long>(b) * D_IDX + part * SC::EPL) * EB);
         // the wpb warps of block j interleave over its row groups
         const int wi = warp % wpb;
-        const uint4 *base = reinterpret_cast<const uint4 *>(k_idx + row0 * D_IDX);
+        const uint4 *base = reinterpret_cast<const uint4 *>(k_idx + row0 * D_IDX * EB);
         const int groups = rw / RPL;  // row groups per warp
         for (int g0 = 0; g0 < groups; g0 += UNR) {
             uint4 ku[UNR];
@@ -112,11 +144,7 @@ __global__ void __launch_bounds__(256) decode_index_scan_kernel(
             }
 #pragma unroll
             for (int u = 0; u < UNR; ++u) {
-                float kf[8];
-                bf16x8_to_f32(ku[u], kf);
-                float sc = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) sc = fmaf(qv[e], kf[e], sc);
+                float sc = qv.dot(ku[u]);
 #pragma unroll
                 for (int o = LPR / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xFFFFFFFFu, sc, o);
                 if (g0 + u < groups) best = fmaxf(best, sc);
@@ -837,33 +865,38 @@ static cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 
 cudaError_t launch_decode_scan(const Shape &sh, const void *q_idx, const void *k_idx,
                                float *block_scores, const PageMap &pm, int *status, int num_sms,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool int8_keys) {
     (void)num_sms;
     const int own = (sh.T - 1) / sh.block;
     if (own > 0) {
-        // 8 warps per CTA; a warp scans at most 64 rows of one block; small
-        // blocks are packed several to a CTA
+        // 8 warps per CTA; a warp scans at most 64 rows of one block (128
+        // rows of int8 keys: the same bytes); small blocks are packed several
+        // to a CTA
+        const int rmax = int8_keys ? 128 : 64;
         int rw, bpc;
         if (sh.block <= 64) {
             rw = sh.block;
             bpc = 8;
-        } else if (sh.block <= 512 && 512 % sh.block == 0) {
-            rw = 64;
-            bpc = 512 / sh.block;
+        } else if (sh.block <= 8 * rmax && (8 * rmax) % sh.block == 0) {
+            rw = rmax;
+            bpc = 8 * rmax / sh.block;
         } else {
             rw = sh.block / 8;
             bpc = 1;
         }
         const long long items = static_cast<long long>(sh.Bt) * own;
         const long long grid = (items + bpc - 1) / bpc;
-        const auto *qi = static_cast<const __nv_bfloat16 *>(q_idx);
-        const auto *ki = static_cast<const __nv_bfloat16 *>(k_idx);
-        if (sh.d_idx == 128)
-            decode_index_scan_kernel<128><<<static_cast<unsigned>(grid), 256, 0, st>>>(
-                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N, rw, bpc, pm, status);
-        else
-            decode_index_scan_kernel<64><<<static_cast<unsigned>(grid), 256, 0, st>>>(
-                qi, ki, block_scores, sh.Bt, sh.T, sh.block, own, sh.N, rw, bpc, pm, status);
+        const dim3 g(static_cast<unsigned>(grid));
+#define MSA_SCAN(DI, SCT)                                                                      \
+    decode_index_scan_kernel<DI, SCT><<<g, 256, 0, st>>>(q_idx, k_idx, block_scores, sh.Bt,   \
+                                                        sh.T, sh.block, own, sh.N, rw, bpc, pm, \
+                                                        status)
+        if (int8_keys) {
+            if (sh.d_idx == 128) MSA_SCAN(128, ScanS8); else MSA_SCAN(64, ScanS8);
+        } else {
+            if (sh.d_idx == 128) MSA_SCAN(128, ScanBf16); else MSA_SCAN(64, ScanBf16);
+        }
+#undef MSA_SCAN
     }
     return cudaGetLastError();
 }

@@ -200,14 +200,36 @@ __device__ __forceinline__ void topk_insert(float (&ts)[CAP], int (&tj)[CAP], fl
     }
 }
 
-template <int D_IDX, int CAP>
+// Index keys as bf16 (kind::f16, fp32 accumulation, K = 16 per MMA) or as
+// signed 8-bit integers (kind::i8, s32 accumulation, K = 32 per MMA: twice
+// the tensor-core rate, and exact for any int8 keys).  A key row of
+// D_IDX * EB bytes is stored as NREG swizzled regions of RP-byte rows:
+// 128-byte swizzle for 128-byte rows, 64-byte swizzle for 64-byte rows.
+template <int D_IDX, int EB>
+struct IndexTile {
+    static constexpr int RB = D_IDX * EB;                  // bytes per key row
+    static constexpr int RP = RB < 128 ? RB : 128;         // bytes per region row
+    static constexpr int NREG = RB / RP;                   // regions per row
+    static constexpr uint32_t QREG = 128u * RP;            // one region of the Q tile
+    static constexpr uint32_t TILE = NREG * QREG;          // Q tile: 128 rows
+    static constexpr uint32_t KREG = kIdxKeys * RP;        // one region of a key tile
+    static constexpr uint32_t KTILE = NREG * KREG;         // key tile: kIdxKeys rows
+    static constexpr int KSTEPS = RB / 32;                 // MMAs per tile (32 bytes of K each)
+    __device__ static uint64_t desc(uint32_t saddr) {
+        return RP == 128 ? sdesc_sw128(saddr, 16, 1024) : sdesc_sw64(saddr);
+    }
+};
+
+template <int D_IDX, int CAP, int EB>
 __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     IndexParams p) {
-    constexpr int NREG = D_IDX / 64;
-    constexpr uint32_t TILE = NREG * kRegionBytes;         // Q tile: 128 rows
-    constexpr uint32_t KREG = kIdxKeys * 128;               // one 64-column region of a key tile
-    constexpr uint32_t KTILE = NREG * KREG;                 // key tile: kIdxKeys rows
+    using TL = IndexTile<D_IDX, EB>;
+    constexpr int NREG = TL::NREG;
+    constexpr uint32_t TILE = TL::TILE;                    // Q tile: 128 rows
+    constexpr uint32_t KREG = TL::KREG;                    // one region of a key tile
+    constexpr uint32_t KTILE = TL::KTILE;                  // key tile: kIdxKeys rows
+    constexpr int XB = TL::RP / EB;                        // TMA box width (elements)
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = align1024(smem_raw);
     unsigned char *q_s = base;
@@ -265,14 +287,14 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
                 if (!mbar_wait(qempty, (it & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
                 mbar_arrive_expect_tx(qfull, TILE);
                 for (int r = 0; r < NREG; ++r)
-                    tma_load_2d(q_s + r * kRegionBytes, &tm_q, qfull, r * 64, b * p.n_q + qt * 128);
+                    tma_load_2d(q_s + r * TL::QREG, &tm_q, qfull, r * XB, b * p.n_q + qt * 128);
                 for (int s = 0; s < n_sub; ++s, ++n) {
                     const uint32_t st = n % kIdxStages, rd = n / kIdxStages;
                     if (!mbar_wait(kempty + st, (rd & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
                     mbar_arrive_expect_tx(kfull + st, KTILE);
                     armed[st] = static_cast<int>(rd & 1);
                     for (int r = 0; r < NREG; ++r)
-                        tma_load_2d(k_s + st * KTILE + r * KREG, &tm_k, kfull + st, r * 64,
+                        tma_load_2d(k_s + st * KTILE + r * KREG, &tm_k, kfull + st, r * XB,
                                     b * p.T + s * kIdxKeys);
                 }
             }
@@ -283,7 +305,8 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, kIdxKeys, false);
+            const uint32_t idesc = EB == 1 ? idesc_s8_s32(128, kIdxKeys)
+                                           : idesc_bf16_f32(128, kIdxKeys, false);
             uint32_t n = 0, acc_n = 0;
             bool ok = true;
             for (int it = 0; ok; ++it) {
@@ -301,11 +324,16 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
                     if (!mbar_wait(tempty + acc, (ar & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t qa = smem_addr(q_s), ka = smem_addr(k_s + st * KTILE);
+                    constexpr int SPR = TL::RP / 32;  // K steps per region row
 #pragma unroll
-                    for (int kk = 0; kk < D_IDX / 16; ++kk) {
-                        const uint32_t koff = (kk % 4) * 32;
-                        umma_bf16(tmem + acc * kIdxKeys, sdesc_sw128(qa + (kk / 4) * kRegionBytes + koff, 16, 1024),
-                                  sdesc_sw128(ka + (kk / 4) * KREG + koff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < TL::KSTEPS; ++kk) {
+                        const uint32_t koff = (kk % SPR) * 32;
+                        const uint64_t ad = TL::desc(qa + (kk / SPR) * TL::QREG + koff);
+                        const uint64_t bd = TL::desc(ka + (kk / SPR) * KREG + koff);
+                        if (EB == 1)
+                            umma_i8(tmem + acc * kIdxKeys, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                        else
+                            umma_bf16(tmem + acc * kIdxKeys, ad, bd, idesc, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(kempty + st);
                     umma_commit(tfull + acc);
@@ -342,25 +370,54 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
                 const uint32_t acc = acc_n & 1, ar = acc_n >> 1;
                 if (!mbar_wait(tfull + acc, ar & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
+                // two halves of 128 columns: four loads in flight, one wait each
+                // (a wait covers every load of the thread), so the load latency
+                // is paid twice per tile rather than once per 32 columns
 #pragma unroll 1
-                for (int c = 0; c < kIdxKeys / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_addr + acc * kIdxKeys + c * 32, v);
-                    tmem_wait_ld();
-                    // block >= 32 and 32 | block: a 32-column chunk lies in one block
-                    float m = -FLT_MAX;
+                for (int h = 0; h < kIdxKeys / 128; ++h) {
+                    uint32_t v[128];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) m = fmaxf(m, __uint_as_float(v[e]));
-                    bm = fmaxf(bm, m);
-                    const int col_end = s * kIdxKeys + c * 32 + 32;
-                    if (col_end % B == 0) {
-                        const int j = col_end / B - 1;
-                        if (j < own) topk_insert<CAP>(ts, tj, bm, j);
-                        bm = -FLT_MAX;
+                    for (int c4 = 0; c4 < 4; ++c4)
+                        tmem_ld32(tmem + lane_addr + acc * kIdxKeys + h * 128 + c4 * 32,
+                                  *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c4));
+                    tmem_wait_ld();
+                    if (h == kIdxKeys / 128 - 1) {  // the accumulator has been read: refill it
+                        tc_fence_before();
+                        mbar_arrive(tempty + acc);
+                    }
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        // block >= 32 and 32 | block: a 32-column chunk lies in one block
+                        float m;
+                        if (EB == 1) {  // s32 accumulators: integer maximum, then exact to fp32
+                            int im = static_cast<int>(v[32 * c4]);
+#pragma unroll
+                            for (int e = 1; e < 32; ++e) im = max(im, static_cast<int>(v[32 * c4 + e]));
+                            m = static_cast<float>(im);
+                        } else {
+                            float g3[3] = {__uint_as_float(v[32 * c4]), __uint_as_float(v[32 * c4 + 1]),
+                                           __uint_as_float(v[32 * c4 + 2])};
+#pragma unroll
+                            for (int e = 3; e + 5 < 32; e += 6) {
+                                g3[0] = fmax3(g3[0], __uint_as_float(v[32 * c4 + e]), __uint_as_float(v[32 * c4 + e + 3]));
+                                g3[1] = fmax3(g3[1], __uint_as_float(v[32 * c4 + e + 1]), __uint_as_float(v[32 * c4 + e + 4]));
+                                g3[2] = fmax3(g3[2], __uint_as_float(v[32 * c4 + e + 2]), __uint_as_float(v[32 * c4 + e + 5]));
+                            }
+                            // columns 27..31 remain
+                            m = fmax3(fmax3(g3[0], g3[1], g3[2]), __uint_as_float(v[32 * c4 + 27]),
+                                      __uint_as_float(v[32 * c4 + 28]));
+                            m = fmax3(m, __uint_as_float(v[32 * c4 + 29]),
+                                      fmaxf(__uint_as_float(v[32 * c4 + 30]), __uint_as_float(v[32 * c4 + 31])));
+                        }
+                        bm = fmaxf(bm, m);
+                        const int col_end = s * kIdxKeys + h * 128 + c4 * 32 + 32;
+                        if (col_end % B == 0) {
+                            const int j = col_end / B - 1;
+                            if (j < own) topk_insert<CAP>(ts, tj, bm, j);
+                            bm = -FLT_MAX;
+                        }
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(tempty + acc);
             }
             if (!ok) break;
             if (valid) {
@@ -439,8 +496,9 @@ struct ItemRows {
 //   warps 0-3 / 4-7: softmax warpgroups SG0 / SG1.  Each takes alternate
 //     128-row chunks of the item: wait for S (which releases the Q tile),
 //     softmax (S -> P in tensor memory), store the rows' lse, hand 1/l to
-//     the epilogue warpgroup, issue PV, wait for it, issue S of its next
-//     chunk.  One elected thread per warpgroup issues that warpgroup's
+//     the epilogue warpgroup, issue PV, then S of its next chunk right
+//     behind it (the MMAs of one thread execute in issue order, so S does
+//     not overwrite P before PV has read it).  One elected thread per warpgroup issues that warpgroup's
 //     tcgen05.mma.
 //   warps 8-11: epilogue warpgroup.  For every chunk in order: read O from
 //     tensor memory (which frees it for the next PV), scale by 1/l, stage
@@ -824,8 +882,11 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
                     issue_pv();
                 }
                 ++pv_n;
-                if (ci + 1 < n) {  // S of the next chunk once PV has read P
-                    if (!wait_role(bar_o + wg, (pv_n - 1) & 1) || !wait_role(q_ready + wg, qr_n & 1)) {
+                if (ci + 1 < n) {
+                    // S of the next chunk overwrites the P that the PV just
+                    // issued reads: tcgen05.mma of one thread execute in
+                    // issue order, so it needs only the next Q tile
+                    if (!wait_role(q_ready + wg, qr_n & 1)) {
                         aborted = true;
                         break;
                     }
@@ -861,7 +922,8 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
 //     buffer).
 //   warp 12 (one thread): streams K and V sub-tiles through a ring of three
 //     tile slots (TMA) and issues every tcgen05.mma: S(x, r, s) once K_s and
-//     (for s = 0) Q of the chunk are in, and PV(x, r, s - 1) has completed;
+//     (for s = 0) Q of the chunk are in -- it may follow PV(x, r, s - 1) at
+//     once, since the MMAs of one thread execute in issue order;
 //     PV(x, r, s) once P is in tensor memory and V_s is in.  A slot is
 //     refilled when every reader of its tile has completed (commit).
 //   warps 13-15: producers, gathering each chunk's Q rows (two halves per
@@ -1244,7 +1306,9 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
                         if (act[x] == 0) {
                             if (!tile_in(tK)) continue;
                             if (ss[x] == 0 && !mbar_test(q_ready + x, mq[x] & 1)) continue;
-                            if ((rr[x] > 0 || ss[x] > 0) && !mbar_test(bar_pv + x, (mp[x] - 1) & 1)) continue;
+                            // S overwrites the P that this warpgroup's previous PV
+                            // reads: that PV was issued earlier by this thread, and
+                            // tcgen05.mma of one thread execute in issue order
                             tc_fence_after();
                             const uint32_t qa = smem_addr(q_s + x * QT);
                             const uint32_t ka = smem_addr(kv_s + ((t0 + tK) % kKvSlots) * kv_tile);
@@ -1360,22 +1424,38 @@ cudaError_t launch_selftest_umma(const CUtensorMap &tm_a, const CUtensorMap &tm_
     return cudaGetLastError();
 }
 
-size_t prefill_index_smem_bytes(int d_idx) {
-    return 1024 + static_cast<size_t>(d_idx / 64) * (kRegionBytes + kIdxStages * kIdxKeys * 128) + 256;
+size_t prefill_index_smem_bytes(int d_idx, int elem_bytes) {
+    const size_t rb = static_cast<size_t>(d_idx) * elem_bytes;  // bytes per key row
+    return 1024 + 128 * rb + kIdxStages * kIdxKeys * rb + 256;
 }
 
-template <int D_IDX, int CAP>
+template <int D_IDX, int CAP, int EB>
 static cudaError_t launch_index_t(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                   const IndexParams &ip, int grid, cudaStream_t st) {
-    const size_t smem = prefill_index_smem_bytes(D_IDX);
-    cudaFuncSetAttribute(prefill_index_kernel<D_IDX, CAP>,
+    const size_t smem = prefill_index_smem_bytes(D_IDX, EB);
+    cudaFuncSetAttribute(prefill_index_kernel<D_IDX, CAP, EB>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    prefill_index_kernel<D_IDX, CAP><<<grid, 192, smem, st>>>(tm_q, tm_k, ip);
+    prefill_index_kernel<D_IDX, CAP, EB><<<grid, 192, smem, st>>>(tm_q, tm_k, ip);
     return cudaGetLastError();
 }
 
+template <int EB>
+static cudaError_t launch_index_eb(const Shape &sh, const CUtensorMap &tm_q,
+                                   const CUtensorMap &tm_k, const IndexParams &ip, int grid,
+                                   cudaStream_t st) {
+    if (sh.d_idx == 128) {
+        if (sh.K <= 8) return launch_index_t<128, 7, EB>(tm_q, tm_k, ip, grid, st);
+        if (sh.K <= 16) return launch_index_t<128, 15, EB>(tm_q, tm_k, ip, grid, st);
+        return launch_index_t<128, 31, EB>(tm_q, tm_k, ip, grid, st);
+    }
+    if (sh.K <= 8) return launch_index_t<64, 7, EB>(tm_q, tm_k, ip, grid, st);
+    if (sh.K <= 16) return launch_index_t<64, 15, EB>(tm_q, tm_k, ip, grid, st);
+    return launch_index_t<64, 31, EB>(tm_q, tm_k, ip, grid, st);
+}
+
 cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                                 int32_t *ids, int *status, int num_sms, cudaStream_t st) {
+                                 int32_t *ids, int *status, int num_sms, cudaStream_t st,
+                                 bool int8_keys) {
     IndexParams ip;
     ip.ids = ids;
     ip.status = status;
@@ -1387,14 +1467,8 @@ cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const
     ip.n_qt = (sh.n_q + 127) / 128;
     ip.n_items = ip.n_qt * sh.Bt;
     const int grid = ip.n_items < num_sms ? ip.n_items : num_sms;
-    if (sh.d_idx == 128) {
-        if (sh.K <= 8) return launch_index_t<128, 7>(tm_q, tm_k, ip, grid, st);
-        if (sh.K <= 16) return launch_index_t<128, 15>(tm_q, tm_k, ip, grid, st);
-        return launch_index_t<128, 31>(tm_q, tm_k, ip, grid, st);
-    }
-    if (sh.K <= 8) return launch_index_t<64, 7>(tm_q, tm_k, ip, grid, st);
-    if (sh.K <= 16) return launch_index_t<64, 15>(tm_q, tm_k, ip, grid, st);
-    return launch_index_t<64, 31>(tm_q, tm_k, ip, grid, st);
+    return int8_keys ? launch_index_eb<1>(sh, tm_q, tm_k, ip, grid, st)
+                     : launch_index_eb<2>(sh, tm_q, tm_k, ip, grid, st);
 }
 
 size_t prefill_attn_smem_bytes(const Shape &sh) {

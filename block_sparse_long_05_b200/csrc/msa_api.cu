@@ -128,16 +128,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 tensor map with 128-byte swizzle; dims/strides innermost first
-// (strides in bytes for dims 1..rank-1).
+// Tensor map (bf16 by default, or bytes) with 128-byte swizzle (or 64-byte
+// for 64-byte box rows); dims/strides innermost first (strides in bytes for
+// dims 1..rank-1).
 bool make_tmap(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
-               const cuuint64_t *strides, const cuuint32_t *box) {
+               const cuuint64_t *strides, const cuuint32_t *box,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
-                          const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const CUresult r = fn(m, dtype, static_cast<cuuint32_t>(rank), const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -170,9 +172,15 @@ msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t *ids, in
                              workspace_bytes, stream, nullptr);
 }
 
-msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids, int Bt, int n_q,
-                             int T, int d_idx, int block, int K, void *workspace,
-                             size_t workspace_bytes, void *stream, const msa_stage_events *ev) {
+}  // extern "C"
+
+namespace {
+
+// Index branch for bf16 (elem_bytes 2) or signed 8-bit (elem_bytes 1) keys.
+msa_status index_topk_impl(const void *q_idx, const void *k_idx, int32_t *ids, int Bt, int n_q,
+                           int T, int d_idx, int block, int K, void *workspace,
+                           size_t workspace_bytes, void *stream, const msa_stage_events *ev,
+                           int elem_bytes) {
     if (!q_idx || !k_idx || !ids) return MSA_ERR_INVALID_ARG;
     Shape sh;
     msa_status s = validate(Bt, n_q, T, 1, 1, 64, d_idx, block, K, true, false, &sh);
@@ -184,10 +192,12 @@ msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids,
     const int sms = num_sms_current();
     if (sms <= 0) return MSA_ERR_CUDA;
     int *status = at<int>(workspace, L.status);
+    const bool s8 = elem_bytes == 1;
     if (n_q == 1) {
         float *scores = at<float>(workspace, L.block_scores);
         mark(ev, 0, true, st);
-        if (launch_decode_scan(sh, q_idx, k_idx, scores, PageMap{}, status, sms, st) != cudaSuccess)
+        if (launch_decode_scan(sh, q_idx, k_idx, scores, PageMap{}, status, sms, st, s8) !=
+            cudaSuccess)
             return MSA_ERR_CUDA;
         mark(ev, 0, false, st);
         mark(ev, 1, true, st);
@@ -195,18 +205,51 @@ msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids,
         mark(ev, 1, false, st);
         return MSA_OK;
     }
+    // key rows of d_idx * elem_bytes bytes, loaded in boxes of at most 128
+    // bytes (64-byte rows use the 64-byte swizzle)
+    const cuuint32_t row_bytes = static_cast<cuuint32_t>(d_idx * elem_bytes);
+    const cuuint32_t box_x = (row_bytes < 128 ? row_bytes : 128) / elem_bytes;
+    const CUtensorMapDataType dt = s8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUtensorMapSwizzle swz = row_bytes < 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     CUtensorMap tq, tk;
     const cuuint64_t dq[2] = {static_cast<cuuint64_t>(d_idx), static_cast<cuuint64_t>(Bt) * n_q};
     const cuuint64_t dk[2] = {static_cast<cuuint64_t>(d_idx), static_cast<cuuint64_t>(Bt) * T};
-    const cuuint64_t str[1] = {static_cast<cuuint64_t>(d_idx) * 2};
-    const cuuint32_t qbox[2] = {64, 128};                              // 128-query tile
-    const cuuint32_t kbox[2] = {64, static_cast<cuuint32_t>(kIdxKeys)};  // key tile
-    if (!make_tmap(&tq, q_idx, 2, dq, str, qbox) || !make_tmap(&tk, k_idx, 2, dk, str, kbox))
+    const cuuint64_t str[1] = {static_cast<cuuint64_t>(row_bytes)};
+    const cuuint32_t qbox[2] = {box_x, 128};                                 // 128-query tile
+    const cuuint32_t kbox[2] = {box_x, static_cast<cuuint32_t>(kIdxKeys)};  // key tile
+    if (!make_tmap(&tq, q_idx, 2, dq, str, qbox, dt, swz) ||
+        !make_tmap(&tk, k_idx, 2, dk, str, kbox, dt, swz))
         return MSA_ERR_CUDA;
     mark(ev, 0, true, st);
-    const cudaError_t e = launch_prefill_index(sh, tq, tk, ids, status, sms, st);
+    const cudaError_t e = launch_prefill_index(sh, tq, tk, ids, status, sms, st, s8);
     mark(ev, 0, false, st);
     return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32_t *ids, int Bt, int n_q,
+                             int T, int d_idx, int block, int K, void *workspace,
+                             size_t workspace_bytes, void *stream, const msa_stage_events *ev) {
+    return index_topk_impl(q_idx, k_idx, ids, Bt, n_q, T, d_idx, block, K, workspace,
+                           workspace_bytes, stream, ev, 2);
+}
+
+msa_status msa_index_topk_i8(const int8_t *q_idx, const int8_t *k_idx, int32_t *ids, int Bt,
+                             int n_q, int T, int d_idx, int block, int K, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    return msa_index_topk_i8_ev(q_idx, k_idx, ids, Bt, n_q, T, d_idx, block, K, workspace,
+                                workspace_bytes, stream, nullptr);
+}
+
+msa_status msa_index_topk_i8_ev(const int8_t *q_idx, const int8_t *k_idx, int32_t *ids, int Bt,
+                                int n_q, int T, int d_idx, int block, int K, void *workspace,
+                                size_t workspace_bytes, void *stream,
+                                const msa_stage_events *ev) {
+    return index_topk_impl(q_idx, k_idx, ids, Bt, n_q, T, d_idx, block, K, workspace,
+                           workspace_bytes, stream, ev, 1);
 }
 
 msa_status msa_select_invert(const int32_t *ids, int32_t *row_ptr, int32_t *entries, int Bt,

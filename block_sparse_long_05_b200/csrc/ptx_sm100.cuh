@@ -213,6 +213,18 @@ __device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tme
         : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::i8 (signed 8-bit integer
+// inputs, s32 accumulation: exact).  One instruction covers K = 32.
+__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on an mbarrier once all previously issued tcgen05.mma of this thread
 // have completed.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
@@ -230,6 +242,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::i8: signed 8-bit A and B, s32 D, M x N tile,
+// both K-major.  Same fields as above with D format 2 (s32) and A / B format
+// 1 (signed 8-bit).
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor for the 128-byte swizzled canonical layouts.
 //   [0,14) start address >> 4; [16,30) leading byte offset >> 4;
 //   [32,46) stride byte offset >> 4; [46,48) version = 1; [61,64) layout = 2
@@ -245,6 +265,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
            (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
            (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
            (2ull << 61);
+}
+
+// The same for K-major 64-byte swizzled layouts (rows of 64 B, 8-row groups
+// SBO = 512 B apart; layout type 4 = SWIZZLE_64B).
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) |
+           (static_cast<uint64_t>(512u >> 4) << 32) | (1ull << 46) | (4ull << 61);
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread (lane) gets its row's 32

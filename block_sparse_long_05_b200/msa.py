@@ -27,7 +27,7 @@ STATUS = {
 EXPORTED = ("msa_workspace_size", "msa_index_topk", "msa_select_invert", "msa_sparse_attn",
             "msa_index_topk_ev", "msa_sparse_attn_ev", "msa_device_status", "msa_status_string",
             "msa_selftest_umma", "msa_sparse_attn_decode_noalloc", "msa_index_topk_paged",
-            "msa_sparse_attn_paged")
+            "msa_sparse_attn_paged", "msa_index_topk_i8", "msa_index_topk_i8_ev")
 
 MAX_STAGES = 4
 
@@ -88,6 +88,10 @@ def load_library(path: str = LIB_PATH):
     lib.msa_status_string.restype = ctypes.c_char_p
     lib.msa_index_topk_ev.argtypes = [P, P, P, I, I, I, I, I, I, P, Z, P, P]
     lib.msa_index_topk_ev.restype = I
+    lib.msa_index_topk_i8.argtypes = [P, P, P, I, I, I, I, I, I, P, Z, P]
+    lib.msa_index_topk_i8.restype = I
+    lib.msa_index_topk_i8_ev.argtypes = [P, P, P, I, I, I, I, I, I, P, Z, P, P]
+    lib.msa_index_topk_i8_ev.restype = I
     lib.msa_sparse_attn_ev.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P, P]
     lib.msa_sparse_attn_ev.restype = I
     lib.msa_sparse_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
@@ -166,6 +170,28 @@ def index_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, block: int, K: int, ws:
                                                    ids.data_ptr(), Bt, n_q, T, d_idx, block, K,
                                                    ws.ptr, ws.nbytes, _stream(stream),
                                                    _stage_events(events)))
+    return ids
+
+
+def index_topk_i8(q_idx: torch.Tensor, k_idx: torch.Tensor, block: int, K: int, ws: Workspace,
+                  ids: torch.Tensor | None = None, stream=None, events=None) -> torch.Tensor:
+    """Index branch on signed 8-bit index keys (msa_index_topk_i8):
+    q_idx [Bt, n_q, d_idx], k_idx [Bt, T, d_idx] int8 -> ids [Bt, n_q, K] int32,
+    the same selection msa_index_topk makes on the same integer values."""
+    _dev(q_idx, torch.int8, "q_idx")
+    _dev(k_idx, torch.int8, "k_idx")
+    Bt, n_q, d_idx = q_idx.shape
+    T = k_idx.shape[1]
+    if k_idx.shape != (Bt, T, d_idx):
+        raise ValueError(f"k_idx shape {tuple(k_idx.shape)} does not match q_idx")
+    if ids is None:
+        ids = torch.empty((Bt, n_q, K), dtype=torch.int32, device=q_idx.device)
+    _dev(ids, torch.int32, "ids")
+    lib = load_library()
+    _check("msa_index_topk_i8", lib.msa_index_topk_i8_ev(q_idx.data_ptr(), k_idx.data_ptr(),
+                                                         ids.data_ptr(), Bt, n_q, T, d_idx, block,
+                                                         K, ws.ptr, ws.nbytes, _stream(stream),
+                                                         _stage_events(events)))
     return ids
 
 

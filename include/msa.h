@@ -102,6 +102,21 @@ MSA_API msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t 
                                   size_t workspace_bytes, void *stream);
 
 /*
+ * Index branch with signed 8-bit index keys: the same selection as
+ * msa_index_topk (same layouts and rules) for q_idx [Bt][n_q][d_idx] and
+ * k_idx [Bt][T][d_idx] stored as int8 instead of bf16.  The pages' index key
+ * is lightweight ([P2 "索引分支"]) and the workloads' keys are small integers,
+ * which int8 holds exactly; the scores are then integer dot products,
+ * computed exactly (prefill: tcgen05 kind::i8 with s32 accumulation, twice
+ * the bf16 tensor-core rate; decode: dp4a over half the bytes of bf16 keys),
+ * so the ids equal those of msa_index_topk on the same integer values.
+ * Keys that are not integers must go through msa_index_topk instead.
+ */
+MSA_API msa_status msa_index_topk_i8(const int8_t *q_idx, const int8_t *k_idx, int32_t *ids,
+                                     int Bt, int n_q, int T, int d_idx, int block, int K,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Selection inversion [P4 section 2.2]: the per-query block lists in ids
  * turned into per-block lists of hit queries, in CSR form over the Bt*N
  * (sequence, block) pairs:
@@ -169,7 +184,8 @@ MSA_API msa_status msa_sparse_attn_paged(const void *q, const void *k_pages, con
  * immediately before (start[i]) and after (stop[i]) the kernels of stage i.
  * Each non-NULL entry must be a cudaEvent_t created on the current device;
  * `events` itself may be NULL.  Stages:
- *   msa_index_topk_ev:  0 = index kernel (prefill) or k_idx scan (decode);
+ *   msa_index_topk_ev, msa_index_topk_i8_ev:
+ *                       0 = index kernel (prefill) or k_idx scan (decode);
  *                       1 = top-K select (decode only).
  *   msa_sparse_attn_ev: 0 = selection inversion (prefill only);
  *                       1 = attention kernel (KV-block-outer or split-K);
@@ -185,6 +201,11 @@ MSA_API msa_status msa_index_topk_ev(const void *q_idx, const void *k_idx, int32
                                      int n_q, int T, int d_idx, int block, int K,
                                      void *workspace, size_t workspace_bytes, void *stream,
                                      const msa_stage_events *events);
+
+MSA_API msa_status msa_index_topk_i8_ev(const int8_t *q_idx, const int8_t *k_idx, int32_t *ids,
+                                        int Bt, int n_q, int T, int d_idx, int block, int K,
+                                        void *workspace, size_t workspace_bytes, void *stream,
+                                        const msa_stage_events *events);
 
 MSA_API msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v,
                                       const int32_t *ids, float *out, float *lse, int Bt,

@@ -86,6 +86,7 @@ def main():
     bench.ClockSampler = FakeClocks
     msa.Workspace = FakeWorkspace
     msa.index_topk = fake_index_topk
+    msa.index_topk_i8 = fake_index_topk
     msa.sparse_attn = fake_sparse_attn
     msa.device_status = lambda ws, stream=None: 0
     W = inputs.Workload

@@ -137,6 +137,17 @@ def test_paged_decode_host_validation(lib):
                1 << 20, None) == 1  # page table not 4-byte aligned
 
 
+def test_index_topk_i8_host_validation(lib):
+    call = lib.msa_index_topk_i8
+    assert call(None, FAKE, FAKE, 1, 8, 8, 64, 64, 4, FAKE, 1 << 20, None) == 1
+    assert call(FAKE, FAKE, FAKE, 1, 9, 8, 64, 64, 4, FAKE, 1 << 20, None) == 1   # n_q > T
+    assert call(FAKE, FAKE, FAKE, 1, 8, 8, 96, 64, 4, FAKE, 1 << 20, None) == 2   # d_idx
+    assert call(FAKE, FAKE, FAKE, 1, 8, 8, 64, 64, 33, FAKE, 1 << 20, None) == 2  # K > 32
+    assert call(FAKE, FAKE, FAKE, 1, 8, 8, 64, 64, 4, FAKE, 16, None) == 3        # ws small
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert call(odd, FAKE, FAKE, 1, 8, 8, 64, 64, 4, FAKE, 1 << 20, None) == 1    # q_idx align
+
+
 def test_select_invert_host_validation(lib):
     call = lib.msa_select_invert
     assert call(None, FAKE, FAKE, 1, 8, 8, 64, 4, FAKE, 1 << 20, None) == 1
