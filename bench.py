@@ -60,6 +60,8 @@ def parse_args(argv=None):
                     help="skip the decode step at each prefill workload's context")
     ap.add_argument("--no-int8", action="store_true",
                     help="skip the variant of each step with the int8 index path")
+    ap.add_argument("--no-paged", action="store_true",
+                    help="skip the paged-KV variant of each decode step")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample (headline)")
     return ap.parse_args(argv)
@@ -244,6 +246,7 @@ class Problem:
             seed = rank_seed(w, rank) if mode == "seq" else w.seed
             self.x = make_inputs(w, device=dev, seed=seed)
         self.int8_index = False  # index branch on int8 copies of the (integer) index keys
+        self.paged = False       # decode through the paged entry points (use_paged)
         self.Hq = (self.hk1 - self.hk0) * w.G
         self.Hkv = self.hk1 - self.hk0
         self.ws = msa.Workspace.for_shape(w.Bt, w.n_q, w.T, self.Hq, self.Hkv, w.d, w.d_idx,
@@ -276,6 +279,12 @@ class Problem:
         x = x or self.x
         y = y or self.y
         ev_idx, ev_attn, ev_gather = ev if ev else (None, None, None)
+        if self.paged:  # decode over a permuted page store (no stage events)
+            msa.index_topk_paged(x["q_idx"], x["k_idx_pages"], x["page_table"], w.T, w.K,
+                                 self.ws, ids=self.ids, stream=stream)
+            msa.sparse_attn_paged(x["q"], x["k_pages"], x["v_pages"], x["page_table"], w.T,
+                                  self.ids, self.ws, out=y["out"], lse=y["lse"], stream=stream)
+            return
         index = msa.index_topk
         qi, ki = x["q_idx"], x["k_idx"]
         if self.int8_index:
@@ -305,6 +314,30 @@ class Problem:
         self.x["k_idx8"] = self.x["k_idx"].to(torch.int8)
         self.int8_index = True
 
+    def use_paged(self, seed=5):
+        """Switch the decode step to the paged entry points: k_idx, K and V
+        scattered block by block into a page store in a seeded random order,
+        with the page table [Bt, N] that maps them back."""
+        import torch
+        w = self.w
+        N = w.n_blocks
+        if not w.is_decode or w.T % w.block:
+            raise ValueError("paged timing covers decode workloads of whole blocks")
+        g = torch.Generator(device=self.dev)
+        g.manual_seed(seed)
+        perm = torch.randperm(w.Bt * N, generator=g, device=self.dev)
+
+        def scatter(t):
+            src = t.view(w.Bt * N, w.block, *t.shape[2:])
+            out = torch.empty_like(src)
+            out[perm] = src
+            return out
+
+        for k in ("k_idx", "k", "v"):
+            self.x[k + "_pages"] = scatter(self.x[k])
+        self.x["page_table"] = perm.view(w.Bt, N).to(torch.int32)
+        self.paged = True
+
     def touched_bytes(self):
         """Bytes one step reads and writes (to decide whether L2 must be
         flushed between timed steps)."""
@@ -312,7 +345,7 @@ class Problem:
         if w.is_decode:
             return sum(decode_bytes(w, self.ids, self.Hq, self.Hkv))
         inputs = sum(t.numel() * t.element_size() for k, t in self.x.items()
-                     if k not in ("q_idx8", "k_idx8"))
+                     if k in ("q", "k", "v", "q_idx", "k_idx"))
         partials = w.Bt * w.n_q * w.K * self.Hq * (w.d * 2 + 4)
         return inputs + partials + self.y["out"].numel() * 4
 
@@ -380,6 +413,8 @@ def measure(prob, steps, warmup, with_e2e):
         raise RuntimeError(f"{w.name}: device status {msa.status_string(st)}")
     # stage times from a second, separate pass (events between the stages
     # would stop consecutive kernels from overlapping their launch)
+    if prob.paged:
+        evs = []
     for ev in evs:
         if flush is not None:
             flush.fill_(1)
@@ -614,6 +649,26 @@ def measure_int8_index(w, prob, r, steps, warmup, peaks, peak_src):
     return obj
 
 
+def measure_paged(w, prob, r, steps, warmup):
+    """The decode step through the paged entry points on a permuted page
+    store (same values, same ids)."""
+    import torch
+    ids_contig = prob.ids.clone()
+    prob.use_paged()
+    try:
+        rp = measure(prob, steps, warmup, False)
+    finally:
+        prob.paged = False
+    obj = {"ms_per_step": rp["ms"], "value": w.Bt / (rp["ms"] / 1e3), "unit": UNIT,
+           "vs_contiguous": r["ms"] / rp["ms"],
+           "ids_equal_contiguous": bool(torch.equal(prob.ids, ids_contig)),
+           "layout": "k_idx, K and V in pages of one block each, scattered in a seeded random "
+                     "order; page table [Bt, N] int32"}
+    for k in ("k_idx_pages", "k_pages", "v_pages", "page_table"):
+        del prob.x[k]
+    return obj
+
+
 def bench_workload(w, args, rank, world, dev, peaks, peak_src, traffic, mode, steps, warmup,
                    with_e2e, decode_at_T, cpu_seconds):
     """Measure one workload; returns its JSON object (the headline's fields
@@ -627,6 +682,10 @@ def bench_workload(w, args, rank, world, dev, peaks, peak_src, traffic, mode, st
     with_i8 = mode == "whole" and not getattr(args, "no_int8", False)
     if with_i8:
         obj_i8 = measure_int8_index(w, prob, r, steps, warmup, peaks, peak_src)
+    with_paged = mode == "whole" and w.is_decode and w.T % w.block == 0 and \
+        not getattr(args, "no_paged", False)
+    if with_paged:
+        obj_paged = measure_paged(w, prob, r, steps, warmup)
     obj = {"workload": w.name, "value": tokens / (r["ms"] / 1e3), "unit": UNIT,
            "ms_per_step": r["ms"], "stage_ms": {k: round(v, 4) for k, v in r["stage_ms"].items()},
            "roofline": roof, "kernels": kernels, "gpu_launches": r["launches"],
@@ -640,6 +699,8 @@ def bench_workload(w, args, rank, world, dev, peaks, peak_src, traffic, mode, st
         obj["attended_pairs"] = r["pairs"]
     if with_i8:
         obj["int8_index"] = obj_i8
+    if with_paged:
+        obj["paged"] = obj_paged
     if "e2e" in r:
         e = r["e2e"]
         obj["e2e"] = {"value": tokens / (e["ms"] / 1e3), "unit": UNIT, "ms_per_step": e["ms"],

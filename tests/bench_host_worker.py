@@ -87,6 +87,11 @@ def main():
     msa.Workspace = FakeWorkspace
     msa.index_topk = fake_index_topk
     msa.index_topk_i8 = fake_index_topk
+    msa.index_topk_paged = lambda q_idx, k_idx_pages, table, T, K, ws, ids=None, stream=None: \
+        fake_index_topk(q_idx, torch.empty((q_idx.shape[0], T, 1)), k_idx_pages.shape[1], K, ws,
+                        ids=ids)
+    msa.sparse_attn_paged = lambda q, kp, vp, table, T, ids, ws, out=None, lse=None, stream=None: \
+        (out, lse)
     msa.sparse_attn = fake_sparse_attn
     msa.device_status = lambda ws, stream=None: 0
     W = inputs.Workload

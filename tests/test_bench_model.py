@@ -99,6 +99,9 @@ def test_bench_line_structure_with_and_without_l2_flush():
             # the same step with the int8 index path, whose ids match the bf16 path's
             assert c["int8_index"]["ids_equal_bf16_path"], name
             assert c["int8_index"]["index_kernel"]["bound"] == exp_bound, name
+            if name.startswith("decode"):  # and through the paged entry points
+                assert c["paged"]["ids_equal_contiguous"], name
+                assert c["paged"]["ms_per_step"] > 0, name
         if mode == "flush":  # fake events tick 0.25 ms per record: one step = 0.25 ms
             assert abs(line["ms_per_step"] - 0.25) < 1e-9
 
