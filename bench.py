@@ -62,6 +62,8 @@ def parse_args(argv=None):
                     help="skip the variant of each step with the int8 index path")
     ap.add_argument("--no-paged", action="store_true",
                     help="skip the paged-KV variant of each decode step")
+    ap.add_argument("--no-min-ws", action="store_true",
+                    help="skip the prefill step with the minimum workspace")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample (headline)")
     return ap.parse_args(argv)
@@ -249,8 +251,11 @@ class Problem:
         self.paged = False       # decode through the paged entry points (use_paged)
         self.Hq = (self.hk1 - self.hk0) * w.G
         self.Hkv = self.hk1 - self.hk0
+        # prefill: the one-pass workspace (all of this rank's kv heads per
+        # attention launch), the fastest choice when the memory is there
+        self.kv_group = None if w.is_decode else self.Hkv
         self.ws = msa.Workspace.for_shape(w.Bt, w.n_q, w.T, self.Hq, self.Hkv, w.d, w.d_idx,
-                                          w.block, w.K, device=dev)
+                                          w.block, w.K, device=dev, kv_group=self.kv_group)
         self.ids = torch.empty((w.Bt, w.n_q, w.K), dtype=torch.int32, device=dev)
         self.y = {"out": torch.empty((w.Bt, w.n_q, self.Hq, w.d), dtype=torch.float32, device=dev),
                   "lse": torch.empty((w.Bt, w.n_q, self.Hq), dtype=torch.float32, device=dev)}
@@ -649,6 +654,23 @@ def measure_int8_index(w, prob, r, steps, warmup, peaks, peak_src):
     return obj
 
 
+def measure_min_workspace(w, prob, r, steps, warmup):
+    """The prefill step with the minimum workspace (msa_workspace_size): the
+    kv heads are attended and merged in groups whose partials fit in it."""
+    from block_sparse_long_05_b200 import msa
+    one = prob.ws
+    prob.ws = msa.Workspace.for_shape(w.Bt, w.n_q, w.T, prob.Hq, prob.Hkv, w.d, w.d_idx,
+                                      w.block, w.K, device=prob.dev)
+    try:
+        rm = measure(prob, steps, warmup, False)
+        nbytes = prob.ws.nbytes
+    finally:
+        prob.ws = one
+    return {"ms_per_step": rm["ms"], "value": w.Bt * w.n_q / (rm["ms"] / 1e3), "unit": UNIT,
+            "workspace_bytes": nbytes, "one_pass_workspace_bytes": one.nbytes,
+            "vs_one_pass": r["ms"] / rm["ms"]}
+
+
 def measure_paged(w, prob, r, steps, warmup):
     """The decode step through the paged entry points on a permuted page
     store (same values, same ids)."""
@@ -686,6 +708,9 @@ def bench_workload(w, args, rank, world, dev, peaks, peak_src, traffic, mode, st
         not getattr(args, "no_paged", False)
     if with_paged:
         obj_paged = measure_paged(w, prob, r, steps, warmup)
+    with_minws = mode == "whole" and not w.is_decode and not getattr(args, "no_min_ws", False)
+    if with_minws:
+        obj_minws = measure_min_workspace(w, prob, r, steps, warmup)
     obj = {"workload": w.name, "value": tokens / (r["ms"] / 1e3), "unit": UNIT,
            "ms_per_step": r["ms"], "stage_ms": {k: round(v, 4) for k, v in r["stage_ms"].items()},
            "roofline": roof, "kernels": kernels, "gpu_launches": r["launches"],
@@ -701,6 +726,8 @@ def bench_workload(w, args, rank, world, dev, peaks, peak_src, traffic, mode, st
         obj["int8_index"] = obj_i8
     if with_paged:
         obj["paged"] = obj_paged
+    if with_minws:
+        obj["min_workspace"] = obj_minws
     if "e2e" in r:
         e = r["e2e"]
         obj["e2e"] = {"value": tokens / (e["ms"] / 1e3), "unit": UNIT, "ms_per_step": e["ms"],

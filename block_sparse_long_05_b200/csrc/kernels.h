@@ -25,13 +25,16 @@ size_t decode_attn_smem_bytes(const Shape &sh);
 cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, const void *v,
                                const int32_t *ids, float *part_o, float *part_lse, int S,
                                const PageMap &pm, int *status, cudaStream_t st, bool pdl);
+// Merges the partials of query heads [h_off, h_off + Hp) (Hp heads per
+// partial row) into those heads of out / lse.  Decode: Hp = Hq, h_off = 0.
 cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            const float *part_lse, const int32_t *ids, float *out, float *lse,
-                           int S, cudaStream_t st, bool pdl);
+                           int S, cudaStream_t st, bool pdl, int Hp = 0, int h_off = 0);
+// counters: [0] items per kv head, then n_cursors work cursors (zeroed).
 cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts,
                           int *pair_totals, int32_t *row_ptr, int32_t *entries, int *item_ptr,
                           AttnItem *items, int *counters, int rows_per_item, int n_chunks,
-                          int *status, cudaStream_t st);
+                          int *status, cudaStream_t st, int n_cursors = 1);
 
 // tcgen05 kernels (kernels_tc.cu)
 size_t selftest_smem_bytes(int N, int Kd);
@@ -46,9 +49,13 @@ cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const
                                  bool int8_keys);
 size_t prefill_attn_smem_bytes(const Shape &sh);
 int prefill_attn_rows_per_item(int G);
+// One launch attends kv heads [hk0, hk0 + nhk) (and their query heads); its
+// partials [rows][K][nhk * G][d] go to part_o / part_lse.  cursor: a zeroed
+// work counter of this launch.
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                 const void *q, const int32_t *row_ptr, const int32_t *entries,
-                                const AttnItem *items, int *counters, void *part_o,
-                                float *part_lse, int *status, int num_sms, cudaStream_t st);
+                                const AttnItem *items, int *counters, int *cursor, int hk0,
+                                int nhk, void *part_o, float *part_lse, int *status, int num_sms,
+                                cudaStream_t st);
 
 }  // namespace msa

@@ -493,7 +493,8 @@ template <typename PT, int D>
 __global__ void __launch_bounds__(256) lse_combine_kernel(
     const PT *__restrict__ part_o, const float *__restrict__ part_lse,
     const int32_t *__restrict__ ids, float *__restrict__ out, float *__restrict__ lse_out, int Hq,
-    int K, int S, int HG, int G, int N) {
+    int K, int S, int HG, int G, int N, int Hp, int h_off) {
+    // partial rows hold Hp heads (query heads h_off .. h_off + Hp - 1 of out)
     grid_dep_wait();  // inputs come from the previous kernel in the stream
     constexpr int VEC = 16 / sizeof(PT);  // elements per 16-byte load
     constexpr int NV = D / VEC;           // 16-byte loads per head row
@@ -508,7 +509,7 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
         const int s = pp / S;
         float l = -INFINITY;
         const int j = ids[row * K + s];
-        if (j >= 0 && j < N) l = part_lse[((row * K + s) * S + pp % S) * Hq + h0 + hh];
+        if (j >= 0 && j < N) l = part_lse[((row * K + s) * S + pp % S) * Hp + h0 + hh];
         wsm[e] = l;
     }
     __syncthreads();
@@ -529,7 +530,7 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
             wsm[pp * HG + hh] = (l == -INFINITY) ? 0.f : exp2f((l - L) * kLog2e);
         }
         Lsm[hh] = L;
-        lse_out[row * Hq + h0 + hh] = L;
+        lse_out[row * Hq + h_off + h0 + hh] = L;
     }
     __syncthreads();
     for (int e = tid; e < HG * NV; e += blockDim.x) {
@@ -542,8 +543,8 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
         const int gh = G > 0 ? ((h0 + hh) & (G - 1)) : 0;
         const int rot = G > 0 ? (gh * (G >= 8 ? 1 : 8 / G)) & 7 : 0;
         const int cr = ((c / VEC) ^ rot) * VEC;
-        const PT *src = part_o + ((row * K) * S * Hq + h0 + hh) * static_cast<long long>(D) + cr;
-        const long long pstride = static_cast<long long>(Hq) * D;  // between consecutive partials
+        const PT *src = part_o + ((row * K) * S * Hp + h0 + hh) * static_cast<long long>(D) + cr;
+        const long long pstride = static_cast<long long>(Hp) * D;  // between consecutive partials
 #pragma unroll 4
         for (int pp = 0; pp < P; ++pp) {
             const float wgt = wsm[pp * HG + hh];
@@ -560,7 +561,7 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(
                 for (int x = 0; x < VEC; ++x) acc[x] += wgt != 0.f ? wgt * f[x] : 0.f;
             }
         }
-        float *dst = out + (row * Hq + h0 + hh) * static_cast<long long>(D) + c;
+        float *dst = out + (row * Hq + h_off + h0 + hh) * static_cast<long long>(D) + c;
 #pragma unroll
         for (int x = 0; x < VEC; x += 4)
             *reinterpret_cast<float4 *>(dst + x) = make_float4(acc[x], acc[x + 1], acc[x + 2], acc[x + 3]);
@@ -723,12 +724,12 @@ __global__ void __launch_bounds__(256) inv_colscan_kernel(int *__restrict__ chun
 
 // Single-CTA exclusive scans: row_ptr over pair totals; item_ptr over
 // ceil(total / rows_per_item) (when items != nullptr); counters[0] = items,
-// counters[1] = 0 (work cursor of the attention kernel).
+// counters[1 .. n_cursors] = 0 (the work cursors of the attention launches).
 __global__ void __launch_bounds__(1024) inv_rowptr_kernel(const int *__restrict__ pair_totals,
                                                            int *__restrict__ row_ptr,
                                                            int *__restrict__ item_ptr,
                                                            int *__restrict__ counters, int n_pairs,
-                                                           int rows_per_item) {
+                                                           int rows_per_item, int n_cursors) {
     __shared__ int ws_a[32], ws_b[32];
     const int per = (n_pairs + blockDim.x - 1) / blockDim.x;
     const int p0 = threadIdx.x * per;
@@ -777,7 +778,7 @@ __global__ void __launch_bounds__(1024) inv_rowptr_kernel(const int *__restrict_
         if (item_ptr) {
             item_ptr[n_pairs] = tb;
             counters[0] = tb;
-            counters[1] = 0;
+            for (int c = 1; c <= n_cursors; ++c) counters[c] = 0;
         }
     }
 }
@@ -940,9 +941,10 @@ cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, co
 
 cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            const float *part_lse, const int32_t *ids, float *out, float *lse,
-                           int S, cudaStream_t st, bool pdl) {
+                           int S, cudaStream_t st, bool pdl, int Hp, int h_off) {
     const long long rows = static_cast<long long>(sh.Bt) * sh.n_q;
-    if (rows * sh.Hq < 4096 && !part_bf16) {
+    if (Hp <= 0) Hp = sh.Hq;
+    if (rows * sh.Hq < 4096 && !part_bf16 && Hp == sh.Hq) {
         // few rows: split the partials of each (row, head) across the warps of a CTA
         int dev = 0, sms = 148;
         if (cudaGetDevice(&dev) == cudaSuccess)
@@ -971,21 +973,21 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
     }
     // heads per CTA: all of them when there are many rows, else fewer so the
     // grid still covers the SMs a few times
-    int HG = sh.Hq;
-    while (HG > 1 && HG % 2 == 0 && rows * (sh.Hq / HG) < 1024) HG /= 2;
+    int HG = Hp;
+    while (HG > 1 && HG % 2 == 0 && rows * (Hp / HG) < 1024) HG /= 2;
     const int vec = part_bf16 ? 8 : 4;
     int threads = HG * sh.d / vec;
     threads = threads > 256 ? 256 : ((threads + 31) / 32) * 32;
     const int P = sh.K * S;
     const size_t smem = static_cast<size_t>(P * HG + HG) * sizeof(float);
-    const dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>(sh.Hq / HG));
+    const dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>(Hp / HG));
 #define MSA_COMBINE(PT, DD)                                                                      \
     do {                                                                                         \
         cudaFuncSetAttribute(lse_combine_kernel<PT, DD>,                                         \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
         e = launch_ex(lse_combine_kernel<PT, DD>, grid, dim3(threads), smem, st, pdl,             \
                       static_cast<const PT *>(part_o), part_lse, ids, out, lse, sh.Hq, sh.K, S,   \
-                      HG, part_bf16 ? sh.G : 0, sh.N);                                            \
+                      HG, part_bf16 ? sh.G : 0, sh.N, Hp, h_off);                                 \
     } while (0)
     cudaError_t e = cudaSuccess;
     if (part_bf16) {
@@ -1000,7 +1002,7 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
 cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts,
                           int *pair_totals, int32_t *row_ptr, int32_t *entries, int *item_ptr,
                           AttnItem *items, int *counters, int rows_per_item, int n_chunks,
-                          int *status, cudaStream_t st) {
+                          int *status, cudaStream_t st, int n_cursors) {
     const size_t hist_bytes = static_cast<size_t>(4) * sh.N * sizeof(int);
     cudaFuncSetAttribute(inv_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(hist_bytes));
@@ -1013,7 +1015,7 @@ cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts
                                                            n_chunks);
     const int n_pairs = sh.Bt * sh.N;
     inv_rowptr_kernel<<<1, 1024, 0, st>>>(pair_totals, row_ptr, item_ptr, counters, n_pairs,
-                                          rows_per_item);
+                                          rows_per_item, n_cursors);
     inv_scatter_kernel<<<cgrid, 128, hist_bytes, st>>>(ids, chunk_counts, row_ptr, entries,
                                                         sh.n_q, sh.K, sh.N, n_chunks, status);
     if (items)

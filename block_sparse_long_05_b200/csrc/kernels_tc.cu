@@ -470,7 +470,10 @@ struct AttnParams {
     const int32_t *row_ptr;
     const int32_t *entries;
     const AttnItem *items;
-    int *counters;  // [0] items per kv head, [1] work cursor
+    int *counters;  // [0] items per kv head
+    int *cursor;    // work cursor of this launch (zero at launch)
+    int hk0, nhk;   // kv heads [hk0, hk0 + nhk) of this launch
+    int Hp;         // heads per partial row (nhk * G): the partial buffer holds this launch's heads
     __nv_bfloat16 *part_o;
     float *part_lse;
     int *status;
@@ -580,7 +583,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     const uint64_t pol_first = l2_policy_evict_first(), pol_last = l2_policy_evict_last();
 
     const int n_items = p.counters[0];
-    const int total = n_items * p.Hkv;
+    const int total = n_items * p.nhk;
     const int G = p.G, TOK = p.TOK, K = p.K;
     const int row = wtid;
     const int tok = row >> p.log2G, g = row & (G - 1);
@@ -707,7 +710,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     auto store_lse = [&](int c, float m_run, float l_run) {
         const int e = tab->entry[c * TOK + tok];
         if (e >= 0) {
-            const long long prow = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G + g;
+            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk - p.hk0) * G + g;
             p.part_lse[prow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2f : -INFINITY;
         }
     };
@@ -764,7 +767,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
             named_barrier(role_bar, 128);
         if (g == 0) {
             if (e >= 0) {
-                const long long prow0 = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G;
+                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk - p.hk0) * G;
                 bulk_store_hint(p.part_o + prow0 * D, stage + tok * tok_bytes, static_cast<uint32_t>(G * D * 2), pol_first);
             }
             bulk_commit();  // one group per chunk (possibly empty) keeps the count in step
@@ -773,12 +776,13 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     };
 
     while (true) {
-        if (tid == 0) *sh_item = atomicAdd(p.counters + 1, 1);
+        if (tid == 0) *sh_item = atomicAdd(p.cursor, 1);
         __syncthreads();
         const int w = *sh_item;
         if (w >= total || *abort_flag) break;
-        const int hk = w / n_items;
-        const AttnItem item = p.items[w - hk * n_items];
+        const int hl = w / n_items;  // kv head of the work index, within this launch
+        const int hk = p.hk0 + hl;
+        const AttnItem item = p.items[w - hl * n_items];
         const int b = item.pair / p.N, j = item.pair - b * p.N;
         cur_j = j;
         cur_hk = hk;
@@ -1009,7 +1013,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
     const uint64_t pol_first = l2_policy_evict_first(), pol_last = l2_policy_evict_last();
 
     const int n_items = p.counters[0];
-    const int total = n_items * p.Hkv;
+    const int total = n_items * p.nhk;
     const int G = p.G, TOK = p.TOK, K = p.K;
     const int row = wtid;
     const int tok = row >> p.log2G, g = row & (G - 1);
@@ -1170,7 +1174,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
         if (wtid == 0) mbar_arrive(o_free + w);
         const int e = tab->entry[c * TOK + tok];
         if (e >= 0) {
-            const long long prow = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G + g;
+            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk - p.hk0) * G + g;
             p.part_lse[prow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
         }
         fence_proxy_async_smem();
@@ -1180,7 +1184,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
             named_barrier(role_bar, 128);
         if (g == 0) {
             if (e >= 0) {
-                const long long prow0 = static_cast<long long>(e) * p.Hq + static_cast<long long>(cur_hk) * G;
+                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk - p.hk0) * G;
                 bulk_store_hint(p.part_o + prow0 * D, st_s + tok * tok_bytes, static_cast<uint32_t>(G * D * 2), pol_first);
             }
             bulk_commit();
@@ -1189,12 +1193,13 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
     };
 
     while (true) {
-        if (tid == 0) *sh_item = atomicAdd(p.counters + 1, 1);
+        if (tid == 0) *sh_item = atomicAdd(p.cursor, 1);
         __syncthreads();
         const int w = *sh_item;
         if (w >= total || *abort_flag) break;
-        const int hk = w / n_items;
-        const AttnItem item = p.items[w - hk * n_items];
+        const int hl = w / n_items;  // kv head of the work index, within this launch
+        const int hk = p.hk0 + hl;
+        const AttnItem item = p.items[w - hl * n_items];
         const int b = item.pair / p.N, j = item.pair - b * p.N;
         cur_j = j;
         cur_hk = hk;
@@ -1489,14 +1494,19 @@ int prefill_attn_rows_per_item(int G) {
 
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                 const void *q, const int32_t *row_ptr, const int32_t *entries,
-                                const AttnItem *items, int *counters, void *part_o,
-                                float *part_lse, int *status, int num_sms, cudaStream_t st) {
+                                const AttnItem *items, int *counters, int *cursor, int hk0,
+                                int nhk, void *part_o, float *part_lse, int *status, int num_sms,
+                                cudaStream_t st) {
     AttnParams ap;
     ap.q = static_cast<const __nv_bfloat16 *>(q);
     ap.row_ptr = row_ptr;
     ap.entries = entries;
     ap.items = items;
     ap.counters = counters;
+    ap.cursor = cursor;
+    ap.hk0 = hk0;
+    ap.nhk = nhk;
+    ap.Hp = nhk * sh.G;
     ap.part_o = static_cast<__nv_bfloat16 *>(part_o);
     ap.part_lse = part_lse;
     ap.status = status;

@@ -50,7 +50,22 @@ msa_status validate(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_idx, i
     return MSA_OK;
 }
 
-WsLayout layout_for(const Shape &sh, bool with_attn) {
+// Prefill partial bytes when kv_group kv heads are attended per launch.
+size_t prefill_partial_bytes(const Shape &sh, int kv_group) {
+    const size_t prow = static_cast<size_t>(sh.Bt) * sh.n_q * sh.K * kv_group * sh.G;
+    return align_up(prow * sh.d * 2, 256) + align_up(prow * 4, 256);
+}
+
+// Largest divisor of Hkv whose partials fit in `budget` bytes (at least 1).
+int kv_group_within(const Shape &sh, size_t budget) {
+    int best = 1;
+    for (int g = 1; g <= sh.Hkv; ++g)
+        if (sh.Hkv % g == 0 && prefill_partial_bytes(sh, g) <= budget) best = g;
+    return best;
+}
+
+// kv_group: prefill kv heads per attention launch (0: all of them).
+WsLayout layout_for(const Shape &sh, bool with_attn, int kv_group = 0) {
     WsLayout L;
     size_t off = 256;  // status word + padding
     auto take = [&](size_t bytes) {
@@ -72,16 +87,17 @@ WsLayout layout_for(const Shape &sh, bool with_attn) {
     L.entries = take(static_cast<size_t>(sh.Bt) * sh.n_q * sh.K * 4);
     L.item_ptr = take(static_cast<size_t>(pairs + 1) * 4);
     L.items = take(static_cast<size_t>(L.max_items) * sizeof(AttnItem));
-    L.counters = take(16);
+    L.counters = take(static_cast<size_t>(2 + sh.Hkv) * 4);  // items, one cursor per launch
     if (with_attn) {
         if (sh.n_q == 1) {
             const size_t prow = static_cast<size_t>(sh.Bt) * sh.K * L.decode_splits;
             L.part_o = take(prow * sh.Hq * sh.d * 4);
             L.part_lse = take(prow * sh.Hq * 4);
         } else {
-            const size_t prow = static_cast<size_t>(sh.Bt) * sh.n_q * sh.K;
-            L.part_o = take(prow * sh.Hq * sh.d * 2);
-            L.part_lse = take(prow * sh.Hq * 4);
+            L.kv_group = kv_group > 0 ? kv_group : sh.Hkv;
+            const size_t prow = static_cast<size_t>(sh.Bt) * sh.n_q * sh.K * L.kv_group * sh.G;
+            L.part_o = take(prow * sh.d * 2);
+            L.part_lse = take(prow * 4);
         }
     }
     L.total = off;
@@ -162,7 +178,15 @@ size_t msa_workspace_size(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_
                           int K) {
     Shape sh;
     if (validate(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K, true, true, &sh) != MSA_OK) return 0;
-    return layout_for(sh, true).total;
+    return layout_for(sh, true, kv_group_within(sh, kPartialBudget)).total;
+}
+
+size_t msa_workspace_size_kv_group(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_idx,
+                                   int block, int K, int kv_group) {
+    Shape sh;
+    if (validate(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K, true, true, &sh) != MSA_OK) return 0;
+    if (kv_group < 1 || Hkv % kv_group != 0) return 0;
+    return layout_for(sh, true, kv_group).total;
 }
 
 msa_status msa_index_topk(const void *q_idx, const void *k_idx, int32_t *ids, int Bt, int n_q,
@@ -291,7 +315,14 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(ids) ||
         !aligned4(lse))
         return MSA_ERR_INVALID_ARG;
-    const WsLayout L = layout_for(sh, true);
+    // prefill: the fewest attention launches (largest kv-head groups) whose
+    // partials fit in the workspace given
+    int group = sh.Hkv;
+    if (n_q > 1) {
+        while (group > 1 && (sh.Hkv % group != 0 || layout_for(sh, true, group).total > workspace_bytes))
+            --group;
+    }
+    const WsLayout L = layout_for(sh, true, group);
     if ((s = check_ws(workspace, workspace_bytes, L)) != MSA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int *status = at<int>(workspace, L.status);
@@ -314,11 +345,12 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     int32_t *ent = at<int32_t>(workspace, L.entries);
     AttnItem *items = at<AttnItem>(workspace, L.items);
     int *counters = at<int>(workspace, L.counters);
+    const int n_launch = sh.Hkv / L.kv_group;
     mark(ev, 0, true, st);
     cudaError_t e = launch_invert(sh, ids, at<int>(workspace, L.chunk_counts),
                                   at<int>(workspace, L.pair_totals), rp, ent,
                                   at<int>(workspace, L.item_ptr), items, counters,
-                                  L.rows_per_item, L.n_chunks, status, st);
+                                  L.rows_per_item, L.n_chunks, status, st, n_launch);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     mark(ev, 0, false, st);
     const int NK = block < 128 ? block : 128;
@@ -331,14 +363,26 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
         return MSA_ERR_CUDA;
     void *po = at<void>(workspace, L.part_o);
     float *pl = at<float>(workspace, L.part_lse);
+    // kv-head groups in turn: attend the group's heads, then merge their
+    // partials into out / lse (the partial buffer holds one group).  With
+    // several groups, the attention stage's events span the combines of all
+    // groups but the last, and the combine stage is the last group's.
     mark(ev, 1, true, st);
-    e = launch_prefill_attn(sh, tk, tv, q, rp, ent, items, counters, po, pl, status, sms, st);
-    if (e != cudaSuccess) return MSA_ERR_CUDA;
-    mark(ev, 1, false, st);
-    mark(ev, 2, true, st);
-    e = launch_combine(sh, po, true, pl, ids, out, lse, 1, st, true);
+    for (int gi = 0; gi < n_launch; ++gi) {
+        const int hk0 = gi * L.kv_group;
+        e = launch_prefill_attn(sh, tk, tv, q, rp, ent, items, counters, counters + 1 + gi, hk0,
+                                L.kv_group, po, pl, status, sms, st);
+        if (e != cudaSuccess) return MSA_ERR_CUDA;
+        if (gi + 1 == n_launch) {
+            mark(ev, 1, false, st);
+            mark(ev, 2, true, st);
+        }
+        e = launch_combine(sh, po, true, pl, ids, out, lse, 1, st, true, L.kv_group * sh.G,
+                           hk0 * sh.G);
+        if (e != cudaSuccess) return MSA_ERR_CUDA;
+    }
     mark(ev, 2, false, st);
-    return cuda_status(e);
+    return MSA_OK;
 }
 
 msa_status msa_index_topk_paged(const void *q_idx, const void *k_idx_pages,

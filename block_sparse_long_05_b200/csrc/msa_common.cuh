@@ -67,6 +67,11 @@ struct WsLayout {
     int max_items = 0;
     int rows_per_item = 0;
     int decode_splits = 0;    // S: splits per block in decode
+    int kv_group = 0;         // prefill: kv heads per attention launch (partials hold their heads)
 };
+
+// Prefill partial buffer size that msa_workspace_size aims under: the kv
+// heads are attended in groups whose partials fit (at least one kv head).
+constexpr size_t kPartialBudget = static_cast<size_t>(4) << 30;
 
 }  // namespace msa

@@ -27,7 +27,8 @@ STATUS = {
 EXPORTED = ("msa_workspace_size", "msa_index_topk", "msa_select_invert", "msa_sparse_attn",
             "msa_index_topk_ev", "msa_sparse_attn_ev", "msa_device_status", "msa_status_string",
             "msa_selftest_umma", "msa_sparse_attn_decode_noalloc", "msa_index_topk_paged",
-            "msa_sparse_attn_paged", "msa_index_topk_i8", "msa_index_topk_i8_ev")
+            "msa_sparse_attn_paged", "msa_index_topk_i8", "msa_index_topk_i8_ev",
+            "msa_workspace_size_kv_group")
 
 MAX_STAGES = 4
 
@@ -76,6 +77,8 @@ def load_library(path: str = LIB_PATH):
     P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.msa_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I]
     lib.msa_workspace_size.restype = Z
+    lib.msa_workspace_size_kv_group.argtypes = [I, I, I, I, I, I, I, I, I, I]
+    lib.msa_workspace_size_kv_group.restype = Z
     lib.msa_index_topk.argtypes = [P, P, P, I, I, I, I, I, I, P, Z, P]
     lib.msa_index_topk.restype = I
     lib.msa_select_invert.argtypes = [P, P, P, I, I, I, I, I, P, Z, P]
@@ -127,8 +130,14 @@ def _dev(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
     return t
 
 
-def workspace_size(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K) -> int:
-    return int(load_library().msa_workspace_size(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K))
+def workspace_size(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K, kv_group=None) -> int:
+    """Workspace bytes: the minimum (msa_workspace_size), or with kv_group
+    the size for prefill attention passes of kv_group kv heads each
+    (kv_group = Hkv: one pass over all heads)."""
+    lib = load_library()
+    if kv_group is None:
+        return int(lib.msa_workspace_size(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K))
+    return int(lib.msa_workspace_size_kv_group(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K, kv_group))
 
 
 class Workspace:
@@ -148,8 +157,9 @@ class Workspace:
         return self.view.data_ptr()
 
     @classmethod
-    def for_shape(cls, Bt, n_q, T, Hq, Hkv, d, d_idx, block, K, device=None) -> "Workspace":
-        return cls(workspace_size(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K), device)
+    def for_shape(cls, Bt, n_q, T, Hq, Hkv, d, d_idx, block, K, device=None,
+                  kv_group=None) -> "Workspace":
+        return cls(workspace_size(Bt, n_q, T, Hq, Hkv, d, d_idx, block, K, kv_group), device)
 
 
 def index_topk(q_idx: torch.Tensor, k_idx: torch.Tensor, block: int, K: int, ws: Workspace,

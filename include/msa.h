@@ -87,9 +87,22 @@ typedef enum msa_status {
  * zero them once before first use (e.g. cudaMemsetAsync(ws, 0, 256)).  The
  * rest is scratch that every call overwrites; two calls that overlap in time
  * must not share a workspace.  Returns 0 for arguments the calls would reject.
+ *
+ * Prefill attention keeps one bf16 partial (and its lse) per (query row,
+ * slot, query head) until the log-sum-exp combine; it attends the kv heads in
+ * groups and merges each group before the next, so the workspace holds one
+ * group's partials.  msa_workspace_size returns the minimum: the largest
+ * group (a divisor of Hkv) whose partials fit in about 4 GiB, at least one kv
+ * head.  Given a larger workspace, msa_sparse_attn uses the largest group that
+ * fits (fewer, longer launches); msa_workspace_size_kv_group gives the size
+ * for kv_group kv heads per pass (kv_group = Hkv: a single pass), or 0 if
+ * kv_group does not divide Hkv.
  */
 MSA_API size_t msa_workspace_size(int Bt, int n_q, int T, int Hq, int Hkv, int d, int d_idx,
                                   int block, int K);
+
+MSA_API size_t msa_workspace_size_kv_group(int Bt, int n_q, int T, int Hq, int Hkv, int d,
+                                           int d_idx, int block, int K, int kv_group);
 
 /*
  * Index branch [P2 "索引分支"]: block max-pooled single-head index scores and
@@ -190,6 +203,10 @@ MSA_API msa_status msa_sparse_attn_paged(const void *q, const void *k_pages, con
  *   msa_sparse_attn_ev: 0 = selection inversion (prefill only);
  *                       1 = attention kernel (KV-block-outer or split-K);
  *                       2 = log-sum-exp combine.
+ *   A prefill that attends its kv heads in several groups (see
+ *   msa_workspace_size) records stage 1 from the first group's attention to
+ *   the last group's, which spans the combines of all groups but the last,
+ *   and stage 2 around the last group's combine.
  */
 #define MSA_MAX_STAGES 4
 typedef struct msa_stage_events {

@@ -55,6 +55,8 @@ class FakeClocks:
 
 
 class FakeWorkspace:
+    nbytes = 1 << 20
+
     @classmethod
     def for_shape(cls, *args, **kwargs):
         return cls()

@@ -44,10 +44,25 @@ def test_workspace_size(lib):
     for w in WORKLOADS.values():
         n = lib.msa_workspace_size(w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K)
         assert n > 0 and n % 256 == 0, w
-    # prefill partials dominate: Bt*n_q*K*Hq*(2d + 4) bytes
-    w = WORKLOADS["prefill_T65536"]
-    n = lib.msa_workspace_size(w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K)
-    assert n >= w.T * w.K * w.Hq * (2 * w.d + 4)
+    # prefill partials dominate: Bt*n_q*K*(heads of one pass)*(2d + 4) bytes; the
+    # minimum holds one kv-head group's partials, the one-pass size all heads'
+    for name in ("prefill_T65536", "long_prefill_T262144"):
+        w = WORKLOADS[name]
+        args = (w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K)
+        n_min = lib.msa_workspace_size(*args)
+        n_one = lib.msa_workspace_size_kv_group(*args, w.Hkv)
+        part = w.T * w.K * w.Hq * (2 * w.d + 4)
+        assert n_one >= part
+        assert n_min <= max(5 << 30, n_one // w.Hkv + (64 << 20))
+        for g in range(1, w.Hkv + 1):
+            n_g = lib.msa_workspace_size_kv_group(*args, g)
+            if w.Hkv % g:
+                assert n_g == 0
+            else:
+                assert n_g >= part * g // w.Hkv and n_g <= n_one
+    w = WORKLOADS["long_prefill_T262144"]
+    assert lib.msa_workspace_size(w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K) \
+        < 5 * 10**9
     # rejected shapes give 0
     assert lib.msa_workspace_size(1, 8, 4, 8, 2, 64, 64, 64, 8) == 0      # n_q > T
     assert lib.msa_workspace_size(1, 8, 64, 8, 3, 64, 64, 64, 8) == 0     # Hq % Hkv

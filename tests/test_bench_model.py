@@ -102,6 +102,8 @@ def test_bench_line_structure_with_and_without_l2_flush():
             if name.startswith("decode"):  # and through the paged entry points
                 assert c["paged"]["ids_equal_contiguous"], name
                 assert c["paged"]["ms_per_step"] > 0, name
+            else:  # and with the minimum (kv-head grouped) workspace
+                assert c["min_workspace"]["ms_per_step"] > 0, name
         if mode == "flush":  # fake events tick 0.25 ms per record: one step = 0.25 ms
             assert abs(line["ms_per_step"] - 0.25) < 1e-9
 

@@ -208,3 +208,25 @@ def test_prefill_ids_beyond_own_and_out_of_range(out_of_range):
         assert msa.device_status(ws) == (6 if out_of_range else 0)
         rows = torch.arange(w.Bt * w.n_q, dtype=torch.int64)
         _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)
+
+
+@pytest.mark.parametrize("w", [SMALL[2], SMALL[3], SMALL[4], SMALL[5]], ids=lambda w: w.name)
+def test_attention_kv_head_groups(w):
+    # workspaces that hold the partials of 1 and of 2 kv heads: the kv heads
+    # are attended and merged group by group; every row must equal the oracle
+    # (and the one-pass result)
+    from block_sparse_long_05_b200 import msa
+    lib_ready()
+    x = make_inputs(w, device="cuda")
+    ids = random_selection(w, device="cuda")
+    one = msa.Workspace.for_shape(w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K,
+                                  kv_group=w.Hkv)
+    ref_out, ref_lse = run_attn(w, x, ids, one)
+    rows = torch.arange(w.Bt * w.n_q, dtype=torch.int64)
+    for g in sorted({1, 2} & {d for d in range(1, w.Hkv + 1) if w.Hkv % d == 0}):
+        ws = msa.Workspace.for_shape(w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K,
+                                     kv_group=g)
+        out, lse = run_attn(w, x, ids, ws)
+        _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)
+        assert torch.allclose(out, ref_out, atol=1e-6, rtol=0) and \
+            torch.allclose(lse, ref_lse, atol=1e-6, rtol=0), f"kv_group {g} differs from one pass"
