@@ -594,7 +594,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     uint32_t pf[2] = {0, 0};                            // producers: q_free phases
     int kv_armed = -1;
     bool aborted = false;
-    int cur_j = 0, cur_hk = 0;
+    int cur_j = 0, cur_hl = 0;  // block and kv head (within this launch) of the item
 
     // bounded wait of the role's thread 0, outcome shared by the role's 128 threads
     auto wait_role = [&](uint64_t *bar, uint32_t parity) -> bool {
@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     auto store_lse = [&](int c, float m_run, float l_run) {
         const int e = tab->entry[c * TOK + tok];
         if (e >= 0) {
-            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk - p.hk0) * G + g;
+            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hl) * G + g;
             p.part_lse[prow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2f : -INFINITY;
         }
     };
@@ -767,7 +767,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
             named_barrier(role_bar, 128);
         if (g == 0) {
             if (e >= 0) {
-                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk - p.hk0) * G;
+                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hl) * G;
                 bulk_store_hint(p.part_o + prow0 * D, stage + tok * tok_bytes, static_cast<uint32_t>(G * D * 2), pol_first);
             }
             bulk_commit();  // one group per chunk (possibly empty) keeps the count in step
@@ -785,7 +785,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
         const AttnItem item = p.items[w - hl * n_items];
         const int b = item.pair / p.N, j = item.pair - b * p.N;
         cur_j = j;
-        cur_hk = hk;
+        cur_hl = hl;
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
@@ -1024,7 +1024,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
     uint32_t mq[2] = {0, 0}, mp[2] = {0, 0}, gt = 0;   // MMA thread: S rounds, PVs, tiles loaded
     uint32_t pf[2] = {0, 0};                           // producers
     bool aborted = false;
-    int cur_j = 0, cur_hk = 0;
+    int cur_j = 0, cur_hl = 0;  // block and kv head (within this launch) of the item
 
     auto wait_role = [&](uint64_t *bar, uint32_t parity) -> bool {
         bool ok = true;
@@ -1174,7 +1174,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
         if (wtid == 0) mbar_arrive(o_free + w);
         const int e = tab->entry[c * TOK + tok];
         if (e >= 0) {
-            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk - p.hk0) * G + g;
+            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hl) * G + g;
             p.part_lse[prow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
         }
         fence_proxy_async_smem();
@@ -1184,7 +1184,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
             named_barrier(role_bar, 128);
         if (g == 0) {
             if (e >= 0) {
-                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk - p.hk0) * G;
+                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hl) * G;
                 bulk_store_hint(p.part_o + prow0 * D, st_s + tok * tok_bytes, static_cast<uint32_t>(G * D * 2), pol_first);
             }
             bulk_commit();
@@ -1202,7 +1202,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
         const AttnItem item = p.items[w - hl * n_items];
         const int b = item.pair / p.N, j = item.pair - b * p.N;
         cur_j = j;
-        cur_hk = hk;
+        cur_hl = hl;
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
