@@ -30,7 +30,8 @@ cudaError_t launch_decode_attn(const Shape &sh, const void *q, const void *k, co
 cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            const float *part_lse, const int32_t *ids, float *out, float *lse,
                            int S, cudaStream_t st, bool pdl, int Hp = 0, int h_off = 0);
-// counters: [0] items per kv head, then n_cursors work cursors (zeroed).
+// counters: n_cursors pairs (items per kv head, a zeroed work cursor), one
+// per attention launch.
 cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts,
                           int *pair_totals, int32_t *row_ptr, int32_t *entries, int *item_ptr,
                           AttnItem *items, int *counters, int rows_per_item, int n_chunks,
@@ -50,12 +51,13 @@ cudaError_t launch_prefill_index(const Shape &sh, const CUtensorMap &tm_q, const
 size_t prefill_attn_smem_bytes(const Shape &sh);
 int prefill_attn_rows_per_item(int G);
 // One launch attends kv heads [hk0, hk0 + nhk) (and their query heads); its
-// partials [rows][K][nhk * G][d] go to part_o / part_lse.  cursor: a zeroed
-// work counter of this launch.
+// partials [rows][K][nhk * G][d] go to part_o / part_lse.  tm_k / tm_v must
+// start at kv head hk0; counters: this launch's pair (items per kv head, a
+// zeroed work cursor).
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                 const void *q, const int32_t *row_ptr, const int32_t *entries,
-                                const AttnItem *items, int *counters, int *cursor, int hk0,
-                                int nhk, void *part_o, float *part_lse, int *status, int num_sms,
+                                const AttnItem *items, int *counters, int hk0, int nhk,
+                                void *part_o, float *part_lse, int *status, int num_sms,
                                 cudaStream_t st);
 
 }  // namespace msa

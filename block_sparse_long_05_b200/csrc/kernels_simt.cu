@@ -723,8 +723,9 @@ __global__ void __launch_bounds__(256) inv_colscan_kernel(int *__restrict__ chun
 }
 
 // Single-CTA exclusive scans: row_ptr over pair totals; item_ptr over
-// ceil(total / rows_per_item) (when items != nullptr); counters[0] = items,
-// counters[1 .. n_cursors] = 0 (the work cursors of the attention launches).
+// ceil(total / rows_per_item) (when items != nullptr); for each attention
+// launch c < n_cursors, counters[2c] = items and counters[2c + 1] = 0 (its
+// work cursor).
 __global__ void __launch_bounds__(1024) inv_rowptr_kernel(const int *__restrict__ pair_totals,
                                                            int *__restrict__ row_ptr,
                                                            int *__restrict__ item_ptr,
@@ -777,8 +778,10 @@ __global__ void __launch_bounds__(1024) inv_rowptr_kernel(const int *__restrict_
         row_ptr[n_pairs] = ta;
         if (item_ptr) {
             item_ptr[n_pairs] = tb;
-            counters[0] = tb;
-            for (int c = 1; c <= n_cursors; ++c) counters[c] = 0;
+            for (int c = 0; c < n_cursors; ++c) {
+                counters[2 * c] = tb;
+                counters[2 * c + 1] = 0;
+            }
         }
     }
 }

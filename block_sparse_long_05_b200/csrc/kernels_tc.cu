@@ -470,14 +470,14 @@ struct AttnParams {
     const int32_t *row_ptr;
     const int32_t *entries;
     const AttnItem *items;
-    int *counters;  // [0] items per kv head
-    int *cursor;    // work cursor of this launch (zero at launch)
-    int hk0, nhk;   // kv heads [hk0, hk0 + nhk) of this launch
-    int Hp;         // heads per partial row (nhk * G): the partial buffer holds this launch's heads
+    int *counters;  // this launch's pair: [0] items per kv head, [1] work cursor
     __nv_bfloat16 *part_o;
     float *part_lse;
     int *status;
-    int Bt, n_q, T, Hq, Hkv, G, block, K, N;
+    int Hq;  // query heads of q (its row stride in heads)
+    int n_q, T;
+    int Hp;  // heads per partial row: this launch's kv heads x G
+    int Hkv, G, block, K, N;
     int NK;      // keys per sub-tile (min(block, 128))
     int NS;      // sub-tiles per block
     int TOK;     // tokens per 128-row chunk = 128 / G
@@ -583,7 +583,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     const uint64_t pol_first = l2_policy_evict_first(), pol_last = l2_policy_evict_last();
 
     const int n_items = p.counters[0];
-    const int total = n_items * p.nhk;
+    const int total = n_items * p.Hkv;
     const int G = p.G, TOK = p.TOK, K = p.K;
     const int row = wtid;
     const int tok = row >> p.log2G, g = row & (G - 1);
@@ -594,7 +594,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     uint32_t pf[2] = {0, 0};                            // producers: q_free phases
     int kv_armed = -1;
     bool aborted = false;
-    int cur_j = 0, cur_hl = 0;  // block and kv head (within this launch) of the item
+    int cur_j = 0, cur_hk = 0;
 
     // bounded wait of the role's thread 0, outcome shared by the role's 128 threads
     auto wait_role = [&](uint64_t *bar, uint32_t parity) -> bool {
@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     auto store_lse = [&](int c, float m_run, float l_run) {
         const int e = tab->entry[c * TOK + tok];
         if (e >= 0) {
-            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hl) * G + g;
+            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk) * G + g;
             p.part_lse[prow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2f : -INFINITY;
         }
     };
@@ -767,7 +767,7 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
             named_barrier(role_bar, 128);
         if (g == 0) {
             if (e >= 0) {
-                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hl) * G;
+                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk) * G;
                 bulk_store_hint(p.part_o + prow0 * D, stage + tok * tok_bytes, static_cast<uint32_t>(G * D * 2), pol_first);
             }
             bulk_commit();  // one group per chunk (possibly empty) keeps the count in step
@@ -776,16 +776,15 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
     };
 
     while (true) {
-        if (tid == 0) *sh_item = atomicAdd(p.cursor, 1);
+        if (tid == 0) *sh_item = atomicAdd(p.counters + 1, 1);
         __syncthreads();
         const int w = *sh_item;
         if (w >= total || *abort_flag) break;
-        const int hl = w / n_items;  // kv head of the work index, within this launch
-        const int hk = p.hk0 + hl;
-        const AttnItem item = p.items[w - hl * n_items];
+        const int hk = w / n_items;
+        const AttnItem item = p.items[w - hk * n_items];
         const int b = item.pair / p.N, j = item.pair - b * p.N;
         cur_j = j;
-        cur_hl = hl;
+        cur_hk = hk;
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
@@ -1013,7 +1012,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
     const uint64_t pol_first = l2_policy_evict_first(), pol_last = l2_policy_evict_last();
 
     const int n_items = p.counters[0];
-    const int total = n_items * p.nhk;
+    const int total = n_items * p.Hkv;
     const int G = p.G, TOK = p.TOK, K = p.K;
     const int row = wtid;
     const int tok = row >> p.log2G, g = row & (G - 1);
@@ -1024,7 +1023,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
     uint32_t mq[2] = {0, 0}, mp[2] = {0, 0}, gt = 0;   // MMA thread: S rounds, PVs, tiles loaded
     uint32_t pf[2] = {0, 0};                           // producers
     bool aborted = false;
-    int cur_j = 0, cur_hl = 0;  // block and kv head (within this launch) of the item
+    int cur_j = 0, cur_hk = 0;
 
     auto wait_role = [&](uint64_t *bar, uint32_t parity) -> bool {
         bool ok = true;
@@ -1174,7 +1173,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
         if (wtid == 0) mbar_arrive(o_free + w);
         const int e = tab->entry[c * TOK + tok];
         if (e >= 0) {
-            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hl) * G + g;
+            const long long prow = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk) * G + g;
             p.part_lse[prow] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2f : -INFINITY;
         }
         fence_proxy_async_smem();
@@ -1184,7 +1183,7 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
             named_barrier(role_bar, 128);
         if (g == 0) {
             if (e >= 0) {
-                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hl) * G;
+                const long long prow0 = static_cast<long long>(e) * p.Hp + static_cast<long long>(cur_hk) * G;
                 bulk_store_hint(p.part_o + prow0 * D, st_s + tok * tok_bytes, static_cast<uint32_t>(G * D * 2), pol_first);
             }
             bulk_commit();
@@ -1193,16 +1192,15 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
     };
 
     while (true) {
-        if (tid == 0) *sh_item = atomicAdd(p.cursor, 1);
+        if (tid == 0) *sh_item = atomicAdd(p.counters + 1, 1);
         __syncthreads();
         const int w = *sh_item;
         if (w >= total || *abort_flag) break;
-        const int hl = w / n_items;  // kv head of the work index, within this launch
-        const int hk = p.hk0 + hl;
-        const AttnItem item = p.items[w - hl * n_items];
+        const int hk = w / n_items;
+        const AttnItem item = p.items[w - hk * n_items];
         const int b = item.pair / p.N, j = item.pair - b * p.N;
         cur_j = j;
-        cur_hl = hl;
+        cur_hk = hk;
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
@@ -1494,27 +1492,26 @@ int prefill_attn_rows_per_item(int G) {
 
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                 const void *q, const int32_t *row_ptr, const int32_t *entries,
-                                const AttnItem *items, int *counters, int *cursor, int hk0,
-                                int nhk, void *part_o, float *part_lse, int *status, int num_sms,
+                                const AttnItem *items, int *counters, int hk0, int nhk,
+                                void *part_o, float *part_lse, int *status, int num_sms,
                                 cudaStream_t st) {
     AttnParams ap;
-    ap.q = static_cast<const __nv_bfloat16 *>(q);
+    // the kernel indexes heads within the launch's group: q starts at the
+    // group's first head (the K/V tensor maps start there too), Hkv counts
+    // the group's kv heads
+    ap.q = static_cast<const __nv_bfloat16 *>(q) + static_cast<size_t>(hk0) * sh.G * sh.d;
     ap.row_ptr = row_ptr;
     ap.entries = entries;
     ap.items = items;
     ap.counters = counters;
-    ap.cursor = cursor;
-    ap.hk0 = hk0;
-    ap.nhk = nhk;
-    ap.Hp = nhk * sh.G;
     ap.part_o = static_cast<__nv_bfloat16 *>(part_o);
     ap.part_lse = part_lse;
     ap.status = status;
-    ap.Bt = sh.Bt;
+    ap.Hp = nhk * sh.G;
     ap.n_q = sh.n_q;
     ap.T = sh.T;
     ap.Hq = sh.Hq;
-    ap.Hkv = sh.Hkv;
+    ap.Hkv = nhk;
     ap.G = sh.G;
     ap.block = sh.block;
     ap.K = sh.K;

@@ -2,6 +2,7 @@
 // validation, workspace layout, TMA tensor maps and kernel dispatch.  No
 // computation happens here; every step of the path runs in the kernels.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -87,7 +88,7 @@ WsLayout layout_for(const Shape &sh, bool with_attn, int kv_group = 0) {
     L.entries = take(static_cast<size_t>(sh.Bt) * sh.n_q * sh.K * 4);
     L.item_ptr = take(static_cast<size_t>(pairs + 1) * 4);
     L.items = take(static_cast<size_t>(L.max_items) * sizeof(AttnItem));
-    L.counters = take(static_cast<size_t>(2 + sh.Hkv) * 4);  // items, one cursor per launch
+    L.counters = take(static_cast<size_t>(2 * sh.Hkv) * 4);  // (items, cursor) per launch
     if (with_attn) {
         if (sh.n_q == 1) {
             const size_t prow = static_cast<size_t>(sh.Bt) * sh.K * L.decode_splits;
@@ -324,6 +325,10 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     }
     const WsLayout L = layout_for(sh, true, group);
     if ((s = check_ws(workspace, workspace_bytes, L)) != MSA_OK) return s;
+    // prefill kernels address a group's partial rows with 32-bit indices
+    // (such a buffer could not fit in device memory anyway: 2^31 x 260 bytes)
+    if (n_q > 1 && static_cast<long long>(Bt) * n_q * K * L.kv_group * sh.G >= (1ll << 31))
+        return MSA_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int *status = at<int>(workspace, L.status);
     if (n_q == 1) {
@@ -354,13 +359,8 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     mark(ev, 0, false, st);
     const int NK = block < 128 ? block : 128;
-    CUtensorMap tk, tv;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Hkv),
-                                static_cast<cuuint64_t>(Bt) * T};
     const cuuint64_t str[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(Hkv) * d * 2};
     const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(NK)};
-    if (!make_tmap(&tk, k, 3, dims, str, box) || !make_tmap(&tv, v, 3, dims, str, box))
-        return MSA_ERR_CUDA;
     void *po = at<void>(workspace, L.part_o);
     float *pl = at<float>(workspace, L.part_lse);
     // kv-head groups in turn: attend the group's heads, then merge their
@@ -370,7 +370,15 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     mark(ev, 1, true, st);
     for (int gi = 0; gi < n_launch; ++gi) {
         const int hk0 = gi * L.kv_group;
-        e = launch_prefill_attn(sh, tk, tv, q, rp, ent, items, counters, counters + 1 + gi, hk0,
+        // K/V tensor maps over this group's kv heads (row stride unchanged)
+        CUtensorMap tk, tv;
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L.kv_group),
+                                    static_cast<cuuint64_t>(Bt) * T};
+        const size_t head_off = static_cast<size_t>(hk0) * d;  // elements
+        if (!make_tmap(&tk, static_cast<const __nv_bfloat16 *>(k) + head_off, 3, dims, str, box) ||
+            !make_tmap(&tv, static_cast<const __nv_bfloat16 *>(v) + head_off, 3, dims, str, box))
+            return MSA_ERR_CUDA;
+        e = launch_prefill_attn(sh, tk, tv, q, rp, ent, items, counters + 2 * gi, hk0,
                                 L.kv_group, po, pl, status, sms, st);
         if (e != cudaSuccess) return MSA_ERR_CUDA;
         if (gi + 1 == n_launch) {
