@@ -95,3 +95,23 @@ def test_decode_many_rows_and_heads():
     # Bt * Hq >= 4096: the combine takes the row-parallel kernel (fp32
     # partials, two splits per 128-key block) instead of the split combine
     _decode_case(Workload("dec_wide", 64, 1, 2048, 64, 8, 128, 128, 4, 64))
+
+
+def test_decode_repeated_calls_one_workspace():
+    # three calls in a row on one workspace, with different selections: each
+    # equals the oracle (the partials of the previous call are never used)
+    from block_sparse_long_05_b200 import msa
+    from oracle import oracle
+    lib_ready()
+    w = Workload("dec_repeat", 6, 1, 5000, 16, 4, 128, 128, 6, 64)
+    x = make_inputs(w, device="cuda")
+    hx = {k: host(v) for k, v in x.items()}
+    ws = msa.Workspace.for_shape(w.Bt, w.n_q, w.T, w.Hq, w.Hkv, w.d, w.d_idx, w.block, w.K)
+    for seed in (3, 4, 5):
+        ids = random_selection(w, device="cuda", seed=seed)
+        out, lse = msa.sparse_attn(x["q"], x["k"], x["v"], ids, w.block, ws)
+        assert msa.device_status(ws) == 0
+        o_ref, l_ref = oracle.sparse_attn(hx["q"], hx["k"], hx["v"], host(ids).reshape(-1, w.K),
+                                          w.Bt, 1, w.T, w.Hq, w.Hkv, w.d, w.block, w.K)
+        assert_close(host(out).numpy().reshape(o_ref.shape), o_ref, f"out (selection {seed})")
+        assert_close(host(lse).numpy().reshape(l_ref.shape), l_ref, f"lse (selection {seed})")
