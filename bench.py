@@ -815,8 +815,10 @@ def run_msa(args, rank, world, local_rank):
         line["clocks"] = head["clocks"]
     if "e2e" in head:
         line["e2e"] = head["e2e"]
-    if "decode_at_T" in head:
-        line["decode_at_T"] = head["decode_at_T"]
+    for key in ("decode_at_T", "int8_index", "paged", "min_workspace", "attended_pairs",
+                "step_bytes", "step_hbm_frac", "step_frac_of_8tbs_nominal"):
+        if key in head:
+            line[key] = head[key]
     if "cpu_baseline" in head:
         line["cpu_baseline"] = head["cpu_baseline"]
     # every workload of the hot path (one GPU): each with its own numbers
