@@ -266,8 +266,13 @@ class Problem:
         w = self.w
         if w.is_decode:  # scan (when there are blocks before own), select, attention, combine
             return (1 if (w.T - 1) // w.block > 0 else 0) + 3
-        # index, 5 inversion kernels, attention, combine
-        return (1 if self.r1 > self.r0 else 0) + 5 + 1 + 1
+        # index, 5 inversion kernels (+3 for the own-block work list when
+        # blocks are longer than 128 keys), per kv-head group the attention
+        # launch(es) and the combine
+        own = w.block > 128
+        groups = self.Hkv // (self.kv_group or self.Hkv)
+        return ((1 if self.r1 > self.r0 else 0) + 5 + (3 if own else 0) +
+                groups * ((2 if own else 1) + 1))
 
     def stage_keys(self):
         w = self.w
@@ -581,6 +586,17 @@ def stage_work(w, prob, pairs):
             "attn2": ("hbm", comb)}
 
 
+def stage_launches(w, prob, stage):
+    """Kernel launches that one stage's event time (and its work and DRAM
+    traffic figures) span: a prefill attention stage runs once per kv-head
+    group, twice per group (hit lists, then each block's own rows) for
+    blocks longer than 128 keys."""
+    if w.is_decode or stage != "attn1":
+        return 1
+    groups = prob.Hkv // (prob.kv_group or prob.Hkv)
+    return groups * (2 if w.block > 128 else 1)
+
+
 def roofline(w, prob, r, peaks, peak_src, traffic):
     """Roofline of the dominant kernel of the step (and of every timed
     stage): achieved = algorithmic work / the stage's event time."""
@@ -610,6 +626,7 @@ def roofline(w, prob, r, peaks, peak_src, traffic):
     roof = {"bound": k["bound"], "kernel": k["kernel"], "achieved": k["achieved"],
             "peak": burst if k["bound"] == "tensor" else hbm, "unit": k["unit"],
             "frac": k["frac"], "traffic": tr, "work_per_launch": k["work_per_launch"],
+            "launches": stage_launches(w, prob, dom),
             "peak_note": (f"bf16 dense burst (cuBLAS, a ms-scale kernel timed alone), of "
                           f"{peak_src}; frac_sustained uses the sustained {sustained} TFLOP/s"
                           if k["bound"] == "tensor" else f"HBM copy bandwidth, of {peak_src}")}

@@ -31,11 +31,13 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
                            const float *part_lse, const int32_t *ids, float *out, float *lse,
                            int S, cudaStream_t st, bool pdl, int Hp = 0, int h_off = 0);
 // counters: n_cursors pairs (items per kv head, a zeroed work cursor), one
-// per attention launch.
+// per attention launch.  own != nullptr: the hit lists leave out each row's
+// own block, and own receives the work list of the own-block pass.
 cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts,
                           int *pair_totals, int32_t *row_ptr, int32_t *entries, int *item_ptr,
                           AttnItem *items, int *counters, int rows_per_item, int n_chunks,
-                          int *status, cudaStream_t st, int n_cursors = 1);
+                          int *status, cudaStream_t st, int n_cursors = 1,
+                          const OwnWork *own = nullptr);
 
 // tcgen05 kernels (kernels_tc.cu)
 size_t selftest_smem_bytes(int N, int Kd);
@@ -54,10 +56,13 @@ int prefill_attn_rows_per_item(int G);
 // partials [rows][K][nhk * G][d] go to part_o / part_lse.  tm_k / tm_v must
 // start at kv head hk0; counters: this launch's pair (items per kv head, a
 // zeroed work cursor).
+// own_ids != nullptr: the own-block pass instead (items: the own rows of each
+// pair): attends each row's own block and writes the partial of the slot
+// that holds it (own_ids: the selection, searched for that slot).
 cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                 const void *q, const int32_t *row_ptr, const int32_t *entries,
                                 const AttnItem *items, int *counters, int hk0, int nhk,
                                 void *part_o, float *part_lse, int *status, int num_sms,
-                                cudaStream_t st);
+                                cudaStream_t st, const int32_t *own_ids = nullptr);
 
 }  // namespace msa

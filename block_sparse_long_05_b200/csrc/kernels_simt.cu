@@ -652,19 +652,24 @@ __global__ void __launch_bounds__(32 * NW) lse_combine_split_kernel(
 // Inversion.  Chunks of kInvRows query rows; warp w of a chunk owns rows
 // [32w, 32w+32).  Per-warp histograms live in shared memory [4][N].
 // ------------------------------------------------------------------------
+// skip_own >= 0: leave out the entries of each row's own block (the block
+// skip_own = block size; own(t) = t / block, t = T - n_q + i), which the
+// own-block pass attends and merges instead.
 __device__ __forceinline__ void warp_histogram(const int32_t *__restrict__ ids, int *hist_w,
                                                int b, int n_q, int K, int N, int row0,
-                                               int *status) {
+                                               int *status, int T, int skip_own) {
     const int lane = threadIdx.x % 32;
     const int i = row0 + lane;
     if (i < n_q) {
         const int32_t *r = ids + (static_cast<long long>(b) * n_q + i) * K;
+        const int own = skip_own > 0 ? (T - n_q + i) / skip_own : -2;
         for (int s = 0; s < K; ++s) {
             const int j = r[s];
-            if (j >= 0 && j < N)
-                atomicAdd(hist_w + j, 1);
-            else if (j != -1 && status)
+            if (j >= 0 && j < N) {
+                if (j != own) atomicAdd(hist_w + j, 1);
+            } else if (j != -1 && status) {
                 atomicOr(status, kDevBadIds);
+            }
         }
     }
 }
@@ -672,13 +677,14 @@ __device__ __forceinline__ void warp_histogram(const int32_t *__restrict__ ids, 
 __global__ void __launch_bounds__(128) inv_count_kernel(const int32_t *__restrict__ ids,
                                                          int *__restrict__ chunk_counts, int n_q,
                                                          int K, int N, int n_chunks,
-                                                         int *__restrict__ status) {
+                                                         int *__restrict__ status, int T,
+                                                         int skip_own) {
     extern __shared__ int hist[];  // [4][N]
     const int chunk = blockIdx.x, b = blockIdx.y;
     for (int e = threadIdx.x; e < 4 * N; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     const int w = threadIdx.x / 32;
-    warp_histogram(ids, hist + w * N, b, n_q, K, N, chunk * kInvRows + 32 * w, status);
+    warp_histogram(ids, hist + w * N, b, n_q, K, N, chunk * kInvRows + 32 * w, status, T, skip_own);
     __syncthreads();
     int *dst = chunk_counts + (static_cast<long long>(b) * n_chunks + chunk) * N;
     for (int j = threadIdx.x; j < N; j += blockDim.x)
@@ -789,14 +795,15 @@ __global__ void __launch_bounds__(1024) inv_rowptr_kernel(const int *__restrict_
 __global__ void __launch_bounds__(128) inv_scatter_kernel(
     const int32_t *__restrict__ ids, const int *__restrict__ chunk_prefix,
     const int *__restrict__ row_ptr, int32_t *__restrict__ entries, int n_q, int K, int N,
-    int n_chunks, int *__restrict__ status) {
+    int n_chunks, int *__restrict__ status, int T, int skip_own) {
     extern __shared__ int hist[];  // [4][N] counts, then cursors
     const int chunk = blockIdx.x, b = blockIdx.y;
     for (int e = threadIdx.x; e < 4 * N; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
     // bad ids were already reported by the count pass
-    warp_histogram(ids, hist + w * N, b, n_q, K, N, chunk * kInvRows + 32 * w, nullptr);
+    warp_histogram(ids, hist + w * N, b, n_q, K, N, chunk * kInvRows + 32 * w, nullptr, T,
+                   skip_own);
     (void)status;
     __syncthreads();
     const int *pre = chunk_prefix + (static_cast<long long>(b) * n_chunks + chunk) * N;
@@ -816,15 +823,28 @@ __global__ void __launch_bounds__(128) inv_scatter_kernel(
         const int i = row0 + r;
         if (i >= n_q) break;
         const long long row = static_cast<long long>(b) * n_q + i;
+        const int own = skip_own > 0 ? (T - n_q + i) / skip_own : -2;
         if (lane < K) {
             const int j = ids[row * K + lane];
-            if (j >= 0 && j < N) {
+            if (j >= 0 && j < N && j != own) {
                 const int pos = atomicAdd(cursor + j, 1);
                 entries[pos] = static_cast<int32_t>(row * K + lane);
             }
         }
         __syncwarp();
     }
+}
+
+// Rows of each (sequence, block) pair whose own block it is: the queries
+// t = T - n_q + i in [j * block, (j + 1) * block).
+__global__ void __launch_bounds__(256) own_totals_kernel(int *__restrict__ own_totals, int n_q,
+                                                          int T, int block, int N, int n_pairs) {
+    const int p = blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= n_pairs) return;
+    const int j = p % N;
+    const long long lo = max(static_cast<long long>(j) * block, static_cast<long long>(T - n_q));
+    const long long hi = min(static_cast<long long>(j + 1) * block, static_cast<long long>(T));
+    own_totals[p] = hi > lo ? static_cast<int>(hi - lo) : 0;
 }
 
 __global__ void __launch_bounds__(256) attn_items_kernel(const int *__restrict__ pair_totals,
@@ -1005,7 +1025,8 @@ cudaError_t launch_combine(const Shape &sh, const void *part_o, bool part_bf16,
 cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts,
                           int *pair_totals, int32_t *row_ptr, int32_t *entries, int *item_ptr,
                           AttnItem *items, int *counters, int rows_per_item, int n_chunks,
-                          int *status, cudaStream_t st, int n_cursors) {
+                          int *status, cudaStream_t st, int n_cursors, const OwnWork *own) {
+    const int skip_own = own ? sh.block : 0;
     const size_t hist_bytes = static_cast<size_t>(4) * sh.N * sizeof(int);
     cudaFuncSetAttribute(inv_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(hist_bytes));
@@ -1013,17 +1034,27 @@ cudaError_t launch_invert(const Shape &sh, const int32_t *ids, int *chunk_counts
                          static_cast<int>(hist_bytes));
     const dim3 cgrid(n_chunks, sh.Bt);
     inv_count_kernel<<<cgrid, 128, hist_bytes, st>>>(ids, chunk_counts, sh.n_q, sh.K, sh.N,
-                                                      n_chunks, status);
+                                                      n_chunks, status, sh.T, skip_own);
     inv_colscan_kernel<<<dim3(sh.N, sh.Bt), 256, 0, st>>>(chunk_counts, pair_totals, sh.N,
                                                            n_chunks);
     const int n_pairs = sh.Bt * sh.N;
     inv_rowptr_kernel<<<1, 1024, 0, st>>>(pair_totals, row_ptr, item_ptr, counters, n_pairs,
                                           rows_per_item, n_cursors);
     inv_scatter_kernel<<<cgrid, 128, hist_bytes, st>>>(ids, chunk_counts, row_ptr, entries,
-                                                        sh.n_q, sh.K, sh.N, n_chunks, status);
+                                                        sh.n_q, sh.K, sh.N, n_chunks, status,
+                                                        sh.T, skip_own);
     if (items)
         attn_items_kernel<<<(n_pairs + 255) / 256, 256, 0, st>>>(pair_totals, item_ptr, items,
                                                                   n_pairs, rows_per_item);
+    if (own) {  // the own-block pass: items over each pair's own rows
+        own_totals_kernel<<<(n_pairs + 255) / 256, 256, 0, st>>>(own->totals, sh.n_q, sh.T,
+                                                                  sh.block, sh.N, n_pairs);
+        inv_rowptr_kernel<<<1, 1024, 0, st>>>(own->totals, own->row_ptr, own->item_ptr,
+                                              own->counters, n_pairs, rows_per_item, n_cursors);
+        attn_items_kernel<<<(n_pairs + 255) / 256, 256, 0, st>>>(own->totals, own->item_ptr,
+                                                                  own->items, n_pairs,
+                                                                  rows_per_item);
+    }
     return cudaGetLastError();
 }
 

@@ -23,6 +23,7 @@
 
 #include <cfloat>
 #include <cstdint>
+#include <type_traits>
 
 #include "kernels.h"
 #include "msa_common.cuh"
@@ -494,6 +495,31 @@ struct ItemRows {
     int t[kItemTokens];           // query position, or -1
 };
 
+// Parameters of the own-block pass: the rows of each block whose own block
+// it is (consecutive queries, causal within the block).  Each row's partial
+// goes to the slot of its selection that holds the own block, as the
+// hit-list pass would have written it; the hit lists leave those entries out.
+struct OwnAttnParams : AttnParams {
+    const int32_t *ids;  // [rows][K] selection (finds the own slot of each row)
+};
+
+// Token table entry of the own-block pass for token k of the own rows of
+// block j: the entry (query row * K + the slot holding j) and position t, or
+// -1 / -1 for a row whose selection does not hold its own block; q offset as
+// in the hit-list pass.
+template <int D>
+__device__ __forceinline__ void own_token(const OwnAttnParams &p, int b, int j, int hk, int k,
+                                          int &e, int &t, int &qo16) {
+    const int t0 = max(j * p.block, p.T - p.n_q);
+    const int qrow = b * p.n_q + (t0 + k - (p.T - p.n_q));
+    int s_own = -1;
+    for (int s = 0; s < p.K; ++s)
+        if (p.ids[static_cast<long long>(qrow) * p.K + s] == j) s_own = s;
+    e = s_own >= 0 ? qrow * p.K + s_own : -1;
+    t = s_own >= 0 ? t0 + k : -1;
+    qo16 = static_cast<int>((static_cast<long long>(qrow) * p.Hq + static_cast<long long>(hk) * p.G) * (D / 8));
+}
+
 // ===========================================================================
 // Prefill attention, K/V block resident (block <= 128): warp-specialised.
 //   warps 0-3 / 4-7: softmax warpgroups SG0 / SG1.  Each takes alternate
@@ -936,10 +962,12 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
 constexpr int kStreamedThreads = 512;
 constexpr int kKvSlots = 3;
 
-template <int D>
+template <int D, typename PT>
 __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-    AttnParams p) {
+    PT p) {
+    // PT = OwnAttnParams: the own-block pass (own rows of each block)
+    constexpr bool OWN = std::is_same<PT, OwnAttnParams>::value;
     constexpr int DREG = D / 64;
     constexpr uint32_t QT = DREG * kRegionBytes;   // Q tile
     constexpr uint32_t STB = QT + 2048;            // staging: 16-byte pad per token
@@ -1204,11 +1232,23 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
         const int list_base = p.row_ptr[item.pair] + item.start;
         const int ntok = item.count;
         const int n_chunks = (ntok + TOK - 1) / TOK;
+        // sub-tiles chunk c attends: all NS, or in the own-block pass those up
+        // to the one holding its last row's position (later keys are masked
+        // for every row of the chunk); non-decreasing in c
+        const int own_off = OWN ? max(j * p.block, p.T - p.n_q) - j * p.block + item.start : 0;
+        auto n_sub = [&](int c) -> int {
+            if constexpr (OWN)
+                return min(NS, (own_off + min((c + 1) * TOK, ntok) - 1) / NK + 1);
+            else
+                return NS;
+        };
 
         for (int i = tid; i < n_chunks * TOK; i += blockDim.x) {
             int e = -1, t = -1;
             int qo16 = 0;
-            if (i < ntok) {
+            if constexpr (OWN) {
+                if (i < ntok) own_token<D>(p, b, j, hk, item.start + i, e, t, qo16);
+            } else if (i < ntok) {
                 e = p.entries[list_base + i];
                 const int qrow = e >= 0 ? e / K : -1;
                 const int bi = qrow >= 0 ? qrow / p.n_q : -1;
@@ -1268,7 +1308,15 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
             if (lane == 0) {
                 const int R = (n_chunks + 1) / 2;              // rounds (chunk pairs)
                 const int nr[2] = {R, n_chunks / 2};           // rounds with a chunk, per warpgroup
-                const int ntiles = R * NS * 2;                 // K_0 V_0 K_1 V_1 ... per round
+                // K_0 V_0 K_1 V_1 ... per round, as many sub-tiles as the
+                // round's later chunk attends
+                int ntiles = R * NS * 2;
+                if constexpr (OWN) {
+                    ntiles = 0;
+                    for (int r = 0; r < R; ++r) ntiles += 2 * n_sub(min(2 * r + 1, n_chunks - 1));
+                }
+                int fr = 0, fs = 0;    // own-block pass: round and sub-tile of the next tile
+                int tb[2] = {0, 0};    // own-block pass: first tile of each warpgroup's round
                 const uint32_t t0 = gt;                        // first tile of the item (global count)
                 int tl = 0;                                    // tiles of the item issued
                 int readers[kKvSlots] = {0, 0, 0};
@@ -1291,20 +1339,34 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
                         const uint32_t gg = t0 + static_cast<uint32_t>(tl);
                         const uint32_t sl = gg % kKvSlots;
                         if (gg < kKvSlots || mbar_test(slot_free + sl, ((gg / kKvSlots) - 1) & 1)) {
-                            const int pair = tl >> 1, s = pair % NS, r = pair / NS;
-                            readers[sl] = (2 * r + 1 < n_chunks) ? 2 : 1;
+                            int s;
+                            if constexpr (OWN) {
+                                s = fs;
+                                readers[sl] = (fs < n_sub(2 * fr) ? 1 : 0) + (2 * fr + 1 < n_chunks ? 1 : 0);
+                            } else {
+                                const int pair = tl >> 1, r = pair / NS;
+                                s = pair % NS;
+                                readers[sl] = (2 * r + 1 < n_chunks) ? 2 : 1;
+                            }
                             unsigned char *dst = kv_s + sl * kv_tile;
                             mbar_arrive_expect_tx(kvfull + sl, kv_tile);
                             const int z = b * p.T + j * p.block + s * NK;
                             for (int rg = 0; rg < DREG; ++rg)
                                 tma_load_3d(dst + rg * NK * 128, (tl & 1) ? &tm_v : &tm_k, kvfull + sl, rg * 64, hk, z);
                             ++tl;
+                            if constexpr (OWN) {
+                                if (!(tl & 1) && ++fs == n_sub(min(2 * fr + 1, n_chunks - 1))) {
+                                    fs = 0;
+                                    ++fr;
+                                }
+                            }
                             progress = true;
                         }
                     }
                     for (int x = 0; x < 2; ++x) {
                         if (rr[x] >= nr[x]) continue;
-                        const int tK = (rr[x] * NS + ss[x]) * 2;
+                        const int tK = OWN ? tb[x] + 2 * ss[x] : (rr[x] * NS + ss[x]) * 2;
+                        const int nsx = n_sub(2 * rr[x] + x);
                         const uint32_t ts = tmem_base + static_cast<uint32_t>(x * 256);
                         if (act[x] == 0) {
                             if (!tile_in(tK)) continue;
@@ -1334,12 +1396,13 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
                                                  sdesc_sw128(va + kk * 16 * 128, static_cast<uint32_t>(NK) * 128, 1024),
                                                  idesc_o, (ss[x] > 0 || kk > 0) ? 1u : 0u);
                             umma_commit(bar_pv + x);
-                            if (ss[x] == NS - 1) umma_commit(bar_o + x);
+                            if (ss[x] == nsx - 1) umma_commit(bar_o + x);
                             release(tK + 1);
                             ++mp[x];
                             act[x] = 0;
-                            if (++ss[x] == NS) {
+                            if (++ss[x] == nsx) {
                                 ss[x] = 0;
+                                if constexpr (OWN) tb[x] += 2 * n_sub(min(2 * rr[x] + 1, n_chunks - 1));
                                 ++rr[x];
                             }
                         }
@@ -1378,17 +1441,18 @@ __global__ void __launch_bounds__(kStreamedThreads, 1) prefill_attn_streamed_ker
             for (int r = 0; r < n && !aborted; ++r) {
                 const int c = wg + 2 * r;
                 float mref = -INFINITY, lsum = 0.f;
-                for (int s = 0; s < NS; ++s) {
+                const int nsc = n_sub(c);
+                for (int s = 0; s < nsc; ++s) {
                     if (!wait_role(bar_s + wg, s_n & 1)) { aborted = true; break; }
                     ++s_n;
-                    if (wtid == 0 && s == NS - 1 && r + 1 < n) mbar_arrive(q_free + wg);
+                    if (wtid == 0 && s == nsc - 1 && r + 1 < n) mbar_arrive(q_free + wg);
                     const bool sok = softmax_sub(c, s, mref, lsum);
                     // the epilogue warpgroup has read O of this warpgroup's previous chunk
                     if (s == 0 && och > 0 && !wait_role(o_free + wg, (och - 1) & 1)) { aborted = true; break; }
-                    if (s == NS - 1) ml_s[wg * 128 + row] = make_float2(mref, lsum);
+                    if (s == nsc - 1) ml_s[wg * 128 + row] = make_float2(mref, lsum);
                     if (named_barrier_or(role_bar, 128, !sok)) { aborted = true; break; }
                     if (wtid == 0) {
-                        if (s == NS - 1) mbar_arrive(ml_ready + wg);
+                        if (s == nsc - 1) mbar_arrive(ml_ready + wg);
                         mbar_arrive(p_ready + wg);
                     }
                     ++pv_n;
@@ -1494,7 +1558,7 @@ cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const 
                                 const void *q, const int32_t *row_ptr, const int32_t *entries,
                                 const AttnItem *items, int *counters, int hk0, int nhk,
                                 void *part_o, float *part_lse, int *status, int num_sms,
-                                cudaStream_t st) {
+                                cudaStream_t st, const int32_t *own_ids) {
     AttnParams ap;
     // the kernel indexes heads within the launch's group: q starts at the
     // group's first head (the K/V tensor maps start there too), Hkv counts
@@ -1523,18 +1587,27 @@ cudaError_t launch_prefill_attn(const Shape &sh, const CUtensorMap &tm_k, const 
     while ((1 << ap.log2G) < sh.G) ++ap.log2G;
     ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(sh.d));
     const size_t smem = prefill_attn_smem_bytes(sh);
-#define MSA_LAUNCH(KERNEL, THREADS)                                                              \
+#define MSA_LAUNCH(KERNEL, THREADS, PARAMS)                                                      \
     do {                                                                                         \
         cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize,                \
                              static_cast<int>(smem));                                            \
-        KERNEL<<<num_sms, THREADS, smem, st>>>(tm_k, tm_v, ap);                                  \
+        KERNEL<<<num_sms, THREADS, smem, st>>>(tm_k, tm_v, PARAMS);                              \
     } while (0)
+    if (own_ids) {  // the own-block pass
+        OwnAttnParams op;
+        static_cast<AttnParams &>(op) = ap;
+        op.ids = own_ids;
+        if (ap.NS == 1) return cudaErrorInvalidValue;  // blocks of one sub-tile have no own pass
+        if (sh.d == 128) MSA_LAUNCH((prefill_attn_streamed_kernel<128, OwnAttnParams>), kStreamedThreads, op);
+        else MSA_LAUNCH((prefill_attn_streamed_kernel<64, OwnAttnParams>), kStreamedThreads, op);
+        return cudaGetLastError();
+    }
     if (ap.NS == 1) {
-        if (sh.d == 128) MSA_LAUNCH(prefill_attn_resident_kernel<128>, kResidentThreads);
-        else MSA_LAUNCH(prefill_attn_resident_kernel<64>, kResidentThreads);
+        if (sh.d == 128) MSA_LAUNCH(prefill_attn_resident_kernel<128>, kResidentThreads, ap);
+        else MSA_LAUNCH(prefill_attn_resident_kernel<64>, kResidentThreads, ap);
     } else {
-        if (sh.d == 128) MSA_LAUNCH(prefill_attn_streamed_kernel<128>, kStreamedThreads);
-        else MSA_LAUNCH(prefill_attn_streamed_kernel<64>, kStreamedThreads);
+        if (sh.d == 128) MSA_LAUNCH((prefill_attn_streamed_kernel<128, AttnParams>), kStreamedThreads, ap);
+        else MSA_LAUNCH((prefill_attn_streamed_kernel<64, AttnParams>), kStreamedThreads, ap);
     }
 #undef MSA_LAUNCH
     return cudaGetLastError();

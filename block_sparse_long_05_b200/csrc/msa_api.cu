@@ -89,6 +89,15 @@ WsLayout layout_for(const Shape &sh, bool with_attn, int kv_group = 0) {
     L.item_ptr = take(static_cast<size_t>(pairs + 1) * 4);
     L.items = take(static_cast<size_t>(L.max_items) * sizeof(AttnItem));
     L.counters = take(static_cast<size_t>(2 * sh.Hkv) * 4);  // (items, cursor) per launch
+    if (with_attn && sh.n_q > 1 && sh.block > 128) {  // the own-block pass's work list
+        L.max_own_items = static_cast<int>((static_cast<long long>(sh.Bt) * sh.n_q + L.rows_per_item - 1) /
+                                               L.rows_per_item + pairs);
+        L.own_totals = take(static_cast<size_t>(pairs) * 4);
+        L.own_row_ptr = take(static_cast<size_t>(pairs + 1) * 4);
+        L.own_item_ptr = take(static_cast<size_t>(pairs + 1) * 4);
+        L.own_items = take(static_cast<size_t>(L.max_own_items) * sizeof(AttnItem));
+        L.own_counters = take(static_cast<size_t>(2 * sh.Hkv) * 4);
+    }
     if (with_attn) {
         if (sh.n_q == 1) {
             const size_t prow = static_cast<size_t>(sh.Bt) * sh.K * L.decode_splits;
@@ -351,11 +360,23 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     AttnItem *items = at<AttnItem>(workspace, L.items);
     int *counters = at<int>(workspace, L.counters);
     const int n_launch = sh.Hkv / L.kv_group;
+    // Blocks of several 128-key sub-tiles: hit lists without each row's own
+    // block, whose rows get their own pass (causal: a chunk of consecutive
+    // rows skips the sub-tiles past its last row).  A single-sub-tile block
+    // has nothing to skip, and its own rows stay in the hit lists.
+    const bool own_pass = block > 128;
+    OwnWork own;
+    own.totals = at<int>(workspace, L.own_totals);
+    own.row_ptr = at<int>(workspace, L.own_row_ptr);
+    own.item_ptr = at<int>(workspace, L.own_item_ptr);
+    own.items = at<AttnItem>(workspace, L.own_items);
+    own.counters = at<int>(workspace, L.own_counters);
     mark(ev, 0, true, st);
     cudaError_t e = launch_invert(sh, ids, at<int>(workspace, L.chunk_counts),
                                   at<int>(workspace, L.pair_totals), rp, ent,
                                   at<int>(workspace, L.item_ptr), items, counters,
-                                  L.rows_per_item, L.n_chunks, status, st, n_launch);
+                                  L.rows_per_item, L.n_chunks, status, st, n_launch,
+                                  own_pass ? &own : nullptr);
     if (e != cudaSuccess) return MSA_ERR_CUDA;
     mark(ev, 0, false, st);
     const int NK = block < 128 ? block : 128;
@@ -363,8 +384,11 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
     const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(NK)};
     void *po = at<void>(workspace, L.part_o);
     float *pl = at<float>(workspace, L.part_lse);
-    // kv-head groups in turn: attend the group's heads, then merge their
-    // partials into out / lse (the partial buffer holds one group).  With
+    // kv-head groups in turn: the hit-list pass attends the selected blocks
+    // (all but the row's own one when there is an own-block pass), the
+    // own-block pass the own blocks; both write per-slot partials (the
+    // partial buffer holds one group), which the combine merges into out /
+    // lse.  With
     // several groups, the attention stage's events span the combines of all
     // groups but the last, and the combine stage is the last group's.
     mark(ev, 1, true, st);
@@ -381,6 +405,12 @@ msa_status msa_sparse_attn_ev(const void *q, const void *k, const void *v, const
         e = launch_prefill_attn(sh, tk, tv, q, rp, ent, items, counters + 2 * gi, hk0,
                                 L.kv_group, po, pl, status, sms, st);
         if (e != cudaSuccess) return MSA_ERR_CUDA;
+        if (own_pass) {
+            e = launch_prefill_attn(sh, tk, tv, q, own.row_ptr, ent, own.items,
+                                    own.counters + 2 * gi, hk0, L.kv_group, po, pl, status, sms,
+                                    st, ids);
+            if (e != cudaSuccess) return MSA_ERR_CUDA;
+        }
         if (gi + 1 == n_launch) {
             mark(ev, 1, false, st);
             mark(ev, 2, true, st);

@@ -45,6 +45,17 @@ struct AttnItem {
 
 inline __host__ __device__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Work list of the own-block pass of the prefill attention: per (sequence,
+// block) pair, the query rows whose own block it is, cut into items like the
+// hit lists (same scans).
+struct OwnWork {
+    int *totals;     // [Bt*N] own rows per pair
+    int *row_ptr;    // [Bt*N + 1] (scan of totals; scratch)
+    int *item_ptr;   // [Bt*N + 1]
+    AttnItem *items; // [max own items]
+    int *counters;   // per attention launch: (items, cursor)
+};
+
 // Workspace layout.  Offsets are in bytes from the workspace base; every
 // region is 256-byte aligned.  Status word at offset 0.
 struct WsLayout {
@@ -58,7 +69,10 @@ struct WsLayout {
     size_t entries = 0;       // int32 [Bt*n_q*K]
     size_t item_ptr = 0;      // int32 [Bt*N + 1]
     size_t items = 0;         // AttnItem [max_items]
-    size_t counters = 0;      // int32 [4]: item count, work cursor
+    size_t counters = 0;      // int32 [2 * launches]: (items per kv head, work cursor)
+    // own-block pass (prefill): own rows per pair, scans, items, counters
+    size_t own_totals = 0, own_row_ptr = 0, own_item_ptr = 0, own_items = 0, own_counters = 0;
+    int max_own_items = 0;
     // attention partials
     size_t part_o = 0;        // prefill: bf16 [Bt*n_q][K][Hq][d]; decode: fp32 [Bt][K*S][Hq][d]
     size_t part_lse = 0;      // fp32 [Bt*n_q][K][Hq]; decode: [Bt][K*S][Hq]

@@ -154,8 +154,11 @@ MSA_API msa_status msa_select_invert(const int32_t *ids, int32_t *row_ptr, int32
  * contributes no key either) and reported as MSA_ERR_BAD_IDS.  Prefill (n_q > 1): inversion, a
  * KV-block-outer tcgen05 kernel that loads each selected KV block into shared
  * memory and gathers its hit queries, then a log-sum-exp combine of the per
- * slot partials.  Decode (n_q == 1): a split-K kernel over the selected blocks,
- * then the same combine.
+ * slot partials.  With blocks longer than 128 keys, each row's own block is
+ * left out of the hit lists and attended by a second, causal launch of the
+ * kernel over the consecutive rows of each block, which skips the 128-key
+ * sub-tiles past each chunk's last row.  Decode (n_q == 1): a split-K kernel
+ * over the selected blocks, then the same combine.
  */
 MSA_API msa_status msa_sparse_attn(const void *q, const void *k, const void *v,
                                    const int32_t *ids, float *out, float *lse, int Bt, int n_q,
@@ -201,7 +204,9 @@ MSA_API msa_status msa_sparse_attn_paged(const void *q, const void *k_pages, con
  *                       0 = index kernel (prefill) or k_idx scan (decode);
  *                       1 = top-K select (decode only).
  *   msa_sparse_attn_ev: 0 = selection inversion (prefill only);
- *                       1 = attention kernel (KV-block-outer or split-K);
+ *                       1 = attention kernel (KV-block-outer: the hit-list
+ *                           launch and, for blocks longer than 128 keys, the
+ *                           own-block launch; or split-K);
  *                       2 = log-sum-exp combine.
  *   A prefill that attends its kv heads in several groups (see
  *   msa_workspace_size) records stage 1 from the first group's attention to

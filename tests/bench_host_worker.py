@@ -101,7 +101,9 @@ def main():
     small = {"tiny_prefill_T4096": W("tiny_prefill_T4096", 1, 128, 128, 8, 2, 64, 32, 4, 64),
              "prefill_T65536": W("prefill_T65536", 1, 256, 256, 8, 2, 64, 32, 4, 64),
              "decode_32x131072": W("decode_32x131072", 3, 1, 2048, 8, 2, 64, 128, 4, 64),
-             "long_prefill_T262144": W("long_prefill_T262144", 1, 256, 256, 8, 2, 64, 64, 4, 64),
+             # blocks of two 128-key sub-tiles, like the 256K prefill's 512
+             "long_prefill_T262144": W("long_prefill_T262144", 1, 1024, 1024, 8, 2, 64, 256, 4,
+                                       64),
              "decode_4x1048576": W("decode_4x1048576", 4, 1, 4096, 8, 2, 64, 128, 4, 64)}
     inputs.WORKLOADS.update(small)
     if sys.argv[1] == "noflush":

@@ -68,6 +68,10 @@ SMALL = [
     Workload("pf_k1", 2, 600, 600, 8, 2, 128, 64, 1, 64),             # own block only
     Workload("pf_chunk", 2, 300, 2000, 8, 2, 64, 128, 6, 64),         # last n_q queries only
     Workload("pf_short", 1, 40, 40, 8, 2, 64, 64, 4, 64),             # single block, T < block
+    # own-block pass with the first own rows mid-block (T - n_q = 2300), Bt = 2
+    Workload("pf_chunk_b512", 2, 700, 3000, 8, 2, 64, 512, 4, 64),
+    # 8 sub-tiles; G = 16 splits each block's 1024 own rows into two work items
+    Workload("pf_b1024_g16", 1, 2500, 2500, 16, 1, 64, 1024, 2, 64),
 ]
 
 
@@ -210,7 +214,8 @@ def test_prefill_ids_beyond_own_and_out_of_range(out_of_range):
         _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)
 
 
-@pytest.mark.parametrize("w", [SMALL[2], SMALL[3], SMALL[4], SMALL[5]], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [SMALL[2], SMALL[3], SMALL[4], SMALL[5], SMALL[10]],
+                         ids=lambda w: w.name)
 def test_attention_kv_head_groups(w):
     # workspaces that hold the partials of 1 and of 2 kv heads: the kv heads
     # are attended and merged group by group; every row must equal the oracle
