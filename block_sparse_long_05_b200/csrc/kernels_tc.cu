@@ -391,9 +391,18 @@ __global__ void __launch_bounds__(192, 1) prefill_index_kernel(
                         // block >= 32 and 32 | block: a 32-column chunk lies in one block
                         float m;
                         if (EB == 1) {  // s32 accumulators: integer maximum, then exact to fp32
-                            int im = static_cast<int>(v[32 * c4]);
+                            // three independent chains of three-input maxima, as below
+                            auto iv = [&](int e) { return static_cast<int>(v[32 * c4 + e]); };
+                            int g3[3] = {iv(0), iv(1), iv(2)};
 #pragma unroll
-                            for (int e = 1; e < 32; ++e) im = max(im, static_cast<int>(v[32 * c4 + e]));
+                            for (int e = 3; e + 5 < 32; e += 6) {
+                                g3[0] = __vimax3_s32(g3[0], iv(e), iv(e + 3));
+                                g3[1] = __vimax3_s32(g3[1], iv(e + 1), iv(e + 4));
+                                g3[2] = __vimax3_s32(g3[2], iv(e + 2), iv(e + 5));
+                            }
+                            // columns 27..31 remain
+                            int im = __vimax3_s32(__vimax3_s32(g3[0], g3[1], g3[2]), iv(27), iv(28));
+                            im = __vimax3_s32(im, iv(29), max(iv(30), iv(31)));
                             m = static_cast<float>(im);
                         } else {
                             float g3[3] = {__uint_as_float(v[32 * c4]), __uint_as_float(v[32 * c4 + 1]),
