@@ -72,6 +72,12 @@ SMALL = [
     Workload("pf_chunk_b512", 2, 700, 3000, 8, 2, 64, 512, 4, 64),
     # 8 sub-tiles; G = 16 splits each block's 1024 own rows into two work items
     Workload("pf_b1024_g16", 1, 2500, 2500, 16, 1, 64, 1024, 2, 64),
+    # own block only: every hit list is empty, the own-block launch does all the work
+    Workload("pf_k1_b256", 2, 900, 900, 8, 2, 64, 256, 1, 64),
+    # K >= N: dense causal over 256-key blocks
+    Workload("pf_dense_b256", 1, 1100, 1100, 8, 2, 128, 256, 8, 128),
+    # d = 128, G = 8, chunked queries over 512-key blocks, own rows from mid-block
+    Workload("pf_chunk_b512_g8", 1, 1500, 4000, 16, 2, 128, 512, 3, 128),
 ]
 
 
@@ -210,6 +216,35 @@ def test_prefill_ids_beyond_own_and_out_of_range(out_of_range):
         ws = _ws(w)
         out, lse = msa.sparse_attn(x["q"], x["k"], x["v"], ids, w.block, ws)
         assert msa.device_status(ws) == (6 if out_of_range else 0)
+        rows = torch.arange(w.Bt * w.n_q, dtype=torch.int64)
+        _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)
+
+
+def _without_own(w, ids):
+    """A copy of a selection in which every other row that also selected an
+    earlier block drops its own block (the slot becomes -1; the own block is
+    the row's largest id, so the row stays ascending)."""
+    h = ids.cpu().clone().view(-1, w.K)
+    for r in range(0, h.shape[0], 2):
+        own = (w.T - w.n_q + r % w.n_q) // w.block
+        row = h[r].tolist()
+        if own in row and any(0 <= j < own for j in row):
+            h[r, row.index(own)] = -1
+    return h.view_as(ids).to(ids.device)
+
+
+def test_prefill_rows_without_own_block():
+    # the selection is the caller's: a row that left out its own block attends
+    # its other blocks only (the own-block launch skips it)
+    from block_sparse_long_05_b200 import msa
+    lib_ready()
+    for w in (Workload("pf_no_own", 1, 1024, 1024, 8, 2, 64, 64, 4, 64),
+              Workload("pf_no_own_b512", 1, 3000, 3000, 8, 4, 128, 512, 3, 64)):
+        x = make_inputs(w, device="cuda")
+        ids = _without_own(w, random_selection(w, device="cuda"))
+        ws = _ws(w)
+        out, lse = msa.sparse_attn(x["q"], x["k"], x["v"], ids, w.block, ws)
+        assert msa.device_status(ws) == 0
         rows = torch.arange(w.Bt * w.n_q, dtype=torch.int64)
         _check_attn(w, x, host(ids).reshape(-1, w.K).numpy(), out, lse, rows)
 
