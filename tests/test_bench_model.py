@@ -140,3 +140,32 @@ def test_bench_head_sharded_prefill_on_two_gloo_ranks():
     for ids_sum, hq, hkv in line["_ranks"]:
         assert ids_sum == line["_ids_sum"]       # the full selection on every rank
         assert hq == line["config"]["Hq"] // 2 and hkv == line["config"]["Hkv"] // 2
+
+
+def test_launch_count_model():
+    """Kernels of the library one step launches, as the C ABI sequences them:
+    prefill = index, 5 inversion kernels (+3 for the own-block work list with
+    blocks longer than 128 keys), then per kv-head group the attention
+    launch(es) (hit lists, own blocks) and the combine; decode = k_idx scan
+    (when a block precedes the query's own), select, attention, combine."""
+    import types
+    count = bench.Problem.launches_per_step.fget
+    W = Workload
+
+    def prob(w, kv_group=None, r0=0, r1=None):
+        return types.SimpleNamespace(w=w, Hkv=w.Hkv, kv_group=kv_group, r0=r0,
+                                     r1=w.n_q if r1 is None else r1)
+
+    small = W("m_b64", 1, 256, 256, 8, 4, 64, 64, 4, 64)
+    wide = W("m_b512", 1, 2048, 2048, 8, 4, 64, 512, 3, 64)
+    assert count(prob(small, kv_group=4)) == 1 + 5 + 1 + 1
+    assert count(prob(wide, kv_group=4)) == 1 + 5 + 3 + 2 + 1
+    assert count(prob(wide, kv_group=2)) == 1 + 5 + 3 + 2 * (2 + 1)
+    assert count(prob(small, kv_group=4, r0=5, r1=5)) == 5 + 1 + 1  # no index rows on this rank
+    assert count(prob(W("m_dec", 2, 1, 300, 8, 4, 64, 64, 4, 64))) == 4
+    assert count(prob(W("m_dec1", 2, 1, 60, 8, 4, 64, 64, 4, 64))) == 3  # own block only: no scan
+    # the attention stage's launches behind its roofline figures
+    assert bench.stage_launches(small, prob(small, kv_group=4), "attn1") == 1
+    assert bench.stage_launches(wide, prob(wide, kv_group=4), "attn1") == 2
+    assert bench.stage_launches(wide, prob(wide, kv_group=2), "attn1") == 4
+    assert bench.stage_launches(wide, prob(wide, kv_group=4), "attn2") == 1
