@@ -652,9 +652,9 @@ __global__ void __launch_bounds__(32 * NW) lse_combine_split_kernel(
 // Inversion.  Chunks of kInvRows query rows; warp w of a chunk owns rows
 // [32w, 32w+32).  Per-warp histograms live in shared memory [4][N].
 // ------------------------------------------------------------------------
-// skip_own >= 0: leave out the entries of each row's own block (the block
-// skip_own = block size; own(t) = t / block, t = T - n_q + i), which the
-// own-block pass attends and merges instead.
+// skip_own > 0 (the block size): leave out the entries of each row's own
+// block (own(t) = t / block, t = T - n_q + i), which the own-block pass
+// attends instead.
 __device__ __forceinline__ void warp_histogram(const int32_t *__restrict__ ids, int *hist_w,
                                                int b, int n_q, int K, int N, int row0,
                                                int *status, int T, int skip_own) {

@@ -967,6 +967,9 @@ __global__ void __launch_bounds__(kResidentThreads, 1) prefill_attn_resident_ker
 //   warps 13-15: producers, gathering each chunk's Q rows (two halves per
 //     tile, registers, evict-last) into the owning warpgroup's Q tile.
 // Tensor memory: SG w owns columns [256w, 256w+256): S/P at +0, O at +128.
+// With OwnAttnParams (the own-block pass) the items are each block's own
+// rows, consecutive queries; a chunk attends only the sub-tiles up to the one
+// holding its last row, and a round loads as many as its later chunk needs.
 // ===========================================================================
 constexpr int kStreamedThreads = 512;
 constexpr int kKvSlots = 3;
