@@ -169,3 +169,22 @@ def test_launch_count_model():
     assert bench.stage_launches(wide, prob(wide, kv_group=4), "attn1") == 2
     assert bench.stage_launches(wide, prob(wide, kv_group=2), "attn1") == 4
     assert bench.stage_launches(wide, prob(wide, kv_group=4), "attn2") == 1
+
+
+def test_dram_traffic_entries_match_the_bench_headlines():
+    """profiles/dram_traffic.json holds a valid entry, keyed as bench.py looks
+    it up (dominant kernel @ workload), for both prefill workloads the bench
+    reports a roofline on, each near or above the stage's algorithmic bytes (q
+    once, K and V once, the bf16 partials with their lse).  The lower bound is
+    0.9 x: partial rows still in the 126 MB L2 when a launch ends reach DRAM
+    after it, and the entries are captures of a smaller case scaled up."""
+    from block_sparse_long_05_b200.inputs import WORKLOADS
+    traffic = bench.load_traffic()
+    for name in ("prefill_T65536", "long_prefill_T262144"):
+        w = WORKLOADS[name]
+        key = f"{bench.kernel_name(w, 'attn1')}@{name}"
+        assert key in traffic, key
+        rows = w.Bt * w.n_q
+        algo = (rows * w.Hq * w.d * 2 + 2 * w.Bt * w.T * w.Hkv * w.d * 2 +
+                rows * w.K * w.Hq * (w.d * 2 + 4))
+        assert 0.9 * algo <= traffic[key] <= 2 * algo, (key, traffic[key], algo)
